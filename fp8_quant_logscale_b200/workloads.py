@@ -1,0 +1,144 @@
+"""Seeded synthetic inputs for the FP8 ICL-attention layer.
+
+This module only draws random numbers; it holds none of the layer's
+arithmetic, so both the CUDA path and the CPU oracle can take their inputs
+from it.  The pages measure on TabArena / OpenML datasets with pretrained
+TabICLv2 and Kumo checkpoints ("[FP8 3/4] Integrate FP8 attention and caching
+into TabICLv2", timing table: 16,384 to 524,288 context rows, 1,024 query
+rows); none of that is available, so these seeded tensors of the same shapes
+stand in for the attention layer's Q/K/V.
+
+Generation recipe (also stated in the design doc): numpy ``Generator(PCG64)``
+streams keyed by (seed, tensor id, chunk index) over 2^22-element chunks,
+standard normal in float32, rounded to fp16 (RNE); per-(tensor, head) factors
+and the 0.1% x20 outliers, where a workload asks for them, come from their own
+streams.  c_h ~ U(0.5, 1.5) fp32 per head; gate g ~ N(0, 1) fp16 per (row, head).
+"""
+from __future__ import annotations
+
+import dataclasses
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+
+_CHUNK = 1 << 22
+_TENSOR_IDS = {"q": 1, "k": 2, "v": 3, "gate": 4, "c_h": 5, "head_factor": 6, "outlier": 7, "queries": 8}
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    n_ctx: int            # N context rows
+    n_query: int          # M query rows
+    heads: int            # H
+    head_dim: int = 64
+    batch: int = 1
+    gated: bool = False   # GatedLogScale with g ~ N(0, 1)
+    head_factor: tuple | None = None   # per-(tensor, head) U(lo, hi) multiplier
+    outliers: float = 0.0  # fraction of elements multiplied by outlier_scale
+    outlier_scale: float = 20.0
+    cached: bool = False   # cached prediction against an n_ctx-row cache
+    seed: int = 0
+    description: str = ""
+
+    @property
+    def rows(self) -> int:
+        return self.n_ctx + self.n_query
+
+
+# The five workloads of the layer's specification, named by what they are.
+WORKLOADS = {
+    "icl_n1k_m128_h4": Workload(
+        "icl_n1k_m128_h4", 1024, 128, 4, seed=1,
+        description="N=1024 context rows, M=128 queries, H=4, d=64, fp16 N(0,1); LogScale n=1024; "
+                    "context self-attention + query->context cross-attention"),
+    "icl_n16k_m1k_h8": Workload(
+        "icl_n16k_m1k_h8", 16384, 1024, 8, head_factor=(0.5, 4.0), seed=2,
+        description="N=16384, M=1024, H=8, d=64, fp16 N(0,1) scaled per (tensor, head) by U(0.5,4); LogScale"),
+    "icl_n128k_m1k_h8_gated": Workload(
+        "icl_n128k_m1k_h8_gated", 131072, 1024, 8, gated=True, outliers=0.001, seed=3,
+        description="N=131072, M=1024, H=8, d=64, fp16 N(0,1) with 0.1% outliers x20; GatedLogScale g~N(0,1)"),
+    "icl_n512k_m1k_h8": Workload(
+        "icl_n512k_m1k_h8", 524288, 1024, 8, seed=4,
+        description="N=524288, M=1024, H=8, d=64, fp16 N(0,1); LogScale; FP8 self + cross attention"),
+    "cached_n512k_m1k_h8": Workload(
+        "cached_n512k_m1k_h8", 524288, 1024, 8, cached=True, seed=5,
+        description="M=1024 fp16 N(0,1) queries, H=8, d=64, LogScale n=524288, against a resident FP8 "
+                    "K/V cache of 524288 rows; equal across query batch splits 1/64/1024"),
+}
+
+
+def _normal_fill(out: np.ndarray, seed: int, tensor: str) -> None:
+    flat = out.reshape(-1)
+    n = flat.size
+    tid = _TENSOR_IDS[tensor]
+
+    def one(ci: int):
+        lo, hi = ci * _CHUNK, min(n, (ci + 1) * _CHUNK)
+        g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, tid, ci])))
+        flat[lo:hi] = g.standard_normal(hi - lo, dtype=np.float32)
+
+    n_chunks = (n + _CHUNK - 1) // _CHUNK
+    if n_chunks <= 2:
+        for ci in range(n_chunks):
+            one(ci)
+    else:
+        with ThreadPoolExecutor(max_workers=8) as ex:
+            list(ex.map(one, range(n_chunks)))
+
+
+def _outliers(x32: np.ndarray, seed: int, tensor_tid: int, frac: float, scale: float) -> None:
+    flat = x32.reshape(-1)
+    n = flat.size
+    for ci in range((n + _CHUNK - 1) // _CHUNK):
+        lo, hi = ci * _CHUNK, min(n, (ci + 1) * _CHUNK)
+        g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, _TENSOR_IDS["outlier"], tensor_tid, ci])))
+        mask = g.random(hi - lo) < frac
+        flat[lo:hi][mask] *= np.float32(scale)
+
+
+def _tensor(w: Workload, tensor: str, shape, seed: int) -> np.ndarray:
+    x = np.empty(shape, np.float32)
+    _normal_fill(x, seed, tensor)
+    if w.head_factor is not None:
+        g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, _TENSOR_IDS["head_factor"],
+                                                                          _TENSOR_IDS[tensor]])))
+        f = g.uniform(w.head_factor[0], w.head_factor[1], size=w.heads).astype(np.float32)
+        x *= f.reshape((1,) * (len(shape) - 2) + (w.heads, 1))
+    if w.outliers > 0:
+        _outliers(x, seed, _TENSOR_IDS[tensor], w.outliers, w.outlier_scale)
+    return x.astype(np.float16)
+
+
+def make_inputs(w: Workload, seed: int | None = None, n_ctx: int | None = None, n_query: int | None = None,
+                heads: int | None = None, batch: int | None = None) -> dict:
+    """Host (numpy) inputs of a workload; sizes may be overridden for small cases.
+
+    Returns q [B,T,H,d] (raw, before query scaling), k, v [B,N,H,d], c_h [H] fp32,
+    gate [B,T,H] fp16 or None, plus the sizes.  For a cached workload the
+    returned q holds the context rows of the fitted layer followed by the M
+    prediction queries, drawn from a separate stream ("queries").
+    """
+    if any(a is not None for a in (n_ctx, n_query, heads, batch)):
+        w = dataclasses.replace(w, n_ctx=n_ctx if n_ctx is not None else w.n_ctx,
+                                n_query=n_query if n_query is not None else w.n_query,
+                                heads=heads if heads is not None else w.heads,
+                                batch=batch if batch is not None else w.batch)
+    s = w.seed if seed is None else seed
+    B, N, M, H, d = w.batch, w.n_ctx, w.n_query, w.heads, w.head_dim
+    q = _tensor(w, "q", (B, N + M, H, d), s)
+    k = _tensor(w, "k", (B, N, H, d), s)
+    v = _tensor(w, "v", (B, N, H, d), s)
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([s, _TENSOR_IDS["c_h"]])))
+    c_h = g.uniform(0.5, 1.5, size=H).astype(np.float32)
+    gate = None
+    if w.gated:
+        gate = np.empty((B, N + M, H), np.float32)
+        _normal_fill(gate, s, "gate")
+        gate = gate.astype(np.float16)
+    out = dict(workload=w, q=q, k=k, v=v, c_h=c_h, gate=gate, B=B, N=N, M=M, H=H, d=d)
+    if w.cached:
+        qq = np.empty((B, M, H, d), np.float32)
+        _normal_fill(qq, s, "queries")
+        out["queries"] = qq.astype(np.float16)
+    return out

@@ -1,0 +1,234 @@
+"""CPU oracle for the FP8 in-context-learning attention layer.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` may import this package; the library under
+``fp8_quant_logscale_b200`` never does.  It shares no code with the CUDA path.
+
+The arithmetic lives in ``oracle.c`` (plain C, OpenMP over rows, built with
+``-O2 -ffp-contract=off`` and no fast-math).  This module only compiles it and
+marshals numpy arrays through ctypes.  Every function is pinned by the
+``-m "not gpu"`` tests against library casts, closed forms, brute force and
+invariants; none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+# KV tile (online-softmax block) and cached-prediction split length that the
+# layer is defined with.  These are algorithm parameters, restated here on the
+# oracle side from the layer's specification (128-key tiles; the cached path
+# cuts the keys into 16384-key chunks whose boundaries depend on N only).
+KV_TILE = 128
+SPLIT_KEYS = 16384
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so (gcc, OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+               "-ffp-contract=off", "-fno-fast-math", "-o", _LIB, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        _declare(_lib)
+    return _lib
+
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I = ctypes.c_int
+_D = ctypes.c_double
+
+
+def _declare(L):
+    L.orc_f16_decode.restype = _D
+    L.orc_f16_decode.argtypes = [ctypes.c_uint16]
+    L.orc_f16_encode.restype = ctypes.c_uint16
+    L.orc_f16_encode.argtypes = [_D]
+    L.orc_e4m3_decode.restype = _D
+    L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+    L.orc_e4m3_encode.restype = ctypes.c_uint8
+    L.orc_e4m3_encode.argtypes = [_D]
+    for name in ("orc_f16_encode_array", "orc_f16_decode_array",
+                 "orc_e4m3_encode_array", "orc_e4m3_decode_array"):
+        getattr(L, name).restype = None
+        getattr(L, name).argtypes = [_P, _I64, _P]
+    L.orc_log_length.restype = ctypes.c_float
+    L.orc_log_length.argtypes = [_I64]
+    L.orc_qscale.restype = None
+    L.orc_qscale.argtypes = [_P, _I, _I64, _I, _I, _I64, _P, _P, _P]
+    L.orc_context_scales.restype = None
+    L.orc_context_scales.argtypes = [_P, _I, _I64, _I64, _I, _I, _P]
+    L.orc_quantize.restype = None
+    L.orc_quantize.argtypes = [_P, _I, _I64, _I, _I, _P, _P]
+    L.orc_attention.restype = None
+    L.orc_attention.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I64, _I64, _I,
+                                _P, _I64, _I64, _I64, _I, _D, _P, _P, _P]
+    L.orc_attention_exact.restype = None
+    L.orc_attention_exact.argtypes = [_P, _P, _P, _I, _I, _I64, _I64, _I, _P, _I64, _P]
+    L.orc_num_threads.restype = _I
+    L.orc_num_threads.argtypes = []
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data
+
+
+def _bits16(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x)
+    return x.view(np.uint16) if x.dtype == np.float16 else x.astype(np.uint16)
+
+
+# --- codecs -----------------------------------------------------------------
+
+def f16_encode(y) -> np.ndarray:
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    out = np.empty(y.shape, np.uint16)
+    lib().orc_f16_encode_array(_ptr(y), y.size, _ptr(out))
+    return out
+
+
+def f16_decode(h) -> np.ndarray:
+    h = _bits16(h)
+    out = np.empty(h.shape, np.float64)
+    lib().orc_f16_decode_array(_ptr(h), h.size, _ptr(out))
+    return out
+
+
+def e4m3_encode(y) -> np.ndarray:
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    out = np.empty(y.shape, np.uint8)
+    lib().orc_e4m3_encode_array(_ptr(y), y.size, _ptr(out))
+    return out
+
+
+def e4m3_decode(c) -> np.ndarray:
+    c = np.ascontiguousarray(c, dtype=np.uint8)
+    out = np.empty(c.shape, np.float64)
+    lib().orc_e4m3_decode_array(_ptr(c), c.size, _ptr(out))
+    return out
+
+
+def log_length(n: int) -> float:
+    return float(lib().orc_log_length(int(n)))
+
+
+def num_threads() -> int:
+    return int(lib().orc_num_threads())
+
+
+# --- the layer ----------------------------------------------------------------
+
+def qscale(q: np.ndarray, n: int, c_h: np.ndarray, gate: np.ndarray | None = None) -> np.ndarray:
+    """LogScale (gate None) or GatedLogScale of q [B, rows, H, d] fp16 -> fp16."""
+    B, rows, H, d = q.shape
+    qb = _bits16(q)
+    c = np.ascontiguousarray(c_h, dtype=np.float32)
+    gb = None if gate is None else _bits16(gate)
+    if gb is not None:
+        assert gb.shape == (B, rows, H)
+    out = np.empty(q.shape, np.uint16)
+    lib().orc_qscale(_ptr(qb), B, rows, H, d, int(n), _ptr(c), _ptr(gb), _ptr(out))
+    return out.view(np.float16)
+
+
+def context_scales(x: np.ndarray, n_ctx: int) -> np.ndarray:
+    """Per-(b, h) scale amax/448 over the first n_ctx rows of x [B, rows, H, d]."""
+    B, rows, H, d = x.shape
+    xb = _bits16(x)
+    out = np.empty((B, H), np.float32)
+    lib().orc_context_scales(_ptr(xb), B, rows, int(n_ctx), H, d, _ptr(out))
+    return out
+
+
+def quantize(x: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """e4m3 codes [B, H, rows, d] of x [B, rows, H, d] / scale[b, h]."""
+    B, rows, H, d = x.shape
+    xb = _bits16(x)
+    s = np.ascontiguousarray(scale, dtype=np.float32).reshape(B, H)
+    out = np.empty((B, H, rows, d), np.uint8)
+    lib().orc_quantize(_ptr(xb), B, rows, H, d, _ptr(s), _ptr(out))
+    return out
+
+
+def attention(q8, k8, v8, s_q, s_k, s_v, rows=None, bc: int = KV_TILE, split: int = 0,
+              quant_p: bool = True, delta: float = 0.0):
+    """FP8 online-softmax attention of the selected rows of q8 to all keys.
+
+    q8 [B,H,T,d], k8/v8 [B,H,N,d] uint8 codes; s_* [B,H] fp32.
+    Returns (out16 [B,n,H,d] fp16, out [B,n,H,d] f64, allowance [B,n,H,d] f64).
+    """
+    q8 = np.ascontiguousarray(q8, np.uint8)
+    k8 = np.ascontiguousarray(k8, np.uint8)
+    v8 = np.ascontiguousarray(v8, np.uint8)
+    B, H, T, d = q8.shape
+    N = k8.shape[2]
+    assert k8.shape == (B, H, N, d) and v8.shape == (B, H, N, d)
+    if rows is None:
+        rows = np.arange(T, dtype=np.int64)
+    rows = np.ascontiguousarray(rows, np.int64)
+    n = rows.size
+    sq = np.ascontiguousarray(s_q, np.float32).reshape(B * H)
+    sk = np.ascontiguousarray(s_k, np.float32).reshape(B * H)
+    sv = np.ascontiguousarray(s_v, np.float32).reshape(B * H)
+    out16 = np.empty((B, n, H, d), np.uint16)
+    out = np.empty((B, n, H, d), np.float64)
+    allow = np.empty((B, n, H, d), np.float64)
+    lib().orc_attention(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv),
+                        B, H, T, N, d, _ptr(rows), n, int(bc), int(split),
+                        1 if quant_p else 0, float(delta),
+                        _ptr(out16), _ptr(out), _ptr(allow))
+    return out16.view(np.float16), out, allow
+
+
+def attention_exact(q, k, v, rows=None):
+    """Double-precision softmax(q k^T / sqrt(d)) v, no quantisation.
+
+    q [B,T,H,d], k/v [B,N,H,d] fp16.  Returns [B,n,H,d] f64.
+    """
+    B, T, H, d = q.shape
+    N = k.shape[1]
+    if rows is None:
+        rows = np.arange(T, dtype=np.int64)
+    rows = np.ascontiguousarray(rows, np.int64)
+    out = np.empty((B, rows.size, H, d), np.float64)
+    lib().orc_attention_exact(_ptr(_bits16(q)), _ptr(_bits16(k)), _ptr(_bits16(v)),
+                              B, H, T, N, d, _ptr(rows), rows.size, _ptr(out))
+    return out
+
+
+def layer(q, k, v, n_ctx: int, c_h, gate=None, rows=None, split: int = 0, delta: float = 0.0):
+    """All steps of the layer on the CPU: qscale -> scales -> e4m3 -> attention.
+
+    q [B,T,H,d] fp16 (T = n_ctx + queries), k/v [B,n_ctx,H,d] fp16.
+    Returns a dict with every intermediate (for staged parity checks).
+    """
+    qs = qscale(q, n_ctx, c_h, gate)
+    s_q = context_scales(qs, n_ctx)
+    s_k = context_scales(k, n_ctx)
+    s_v = context_scales(v, n_ctx)
+    q8 = quantize(qs, s_q)
+    k8 = quantize(k, s_k)
+    v8 = quantize(v, s_v)
+    o16, o, allow = attention(q8, k8, v8, s_q, s_k, s_v, rows=rows, split=split, delta=delta)
+    return dict(q_scaled=qs, s_q=s_q, s_k=s_k, s_v=s_v, q8=q8, k8=k8, v8=v8,
+                out16=o16, out=o, allow=allow)

@@ -1,0 +1,184 @@
+"""Pins of the oracle's FP8 attention and cached (split-KV) prediction (CPU only).
+
+Against: a naive full-row double softmax (quantisation of P switched off), a
+materialised-P implementation in numpy + torch's e4m3 cast, a hand-worked
+golden example with exact powers of two, Q = 0 (mean of V), constant V (the
+row sum normalises), permutation of the context rows, partitions of the query
+batch for the cached path, and the pages' block-level accuracy bound against
+exact attention ("[FP8 4/5]" KumoTabular page, review of
+test/models/test_attention_quantization.py: relative RMS < 0.08).
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from fp8_quant_logscale_b200.workloads import WORKLOADS, make_inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+LOG2E = 1.4426950408889634
+
+
+def _codes(orc, B, H, rows, seed, scale=1.0):
+    rng = np.random.default_rng(seed)
+    x = (rng.standard_normal((B, rows, H, 64)) * scale).astype(np.float16)
+    s = orc.context_scales(x, rows)
+    return orc.quantize(x, s), s
+
+
+def _problem(orc, B=1, H=2, T=40, N=300, seed=0, qscale=0.4):
+    q8, sq = _codes(orc, B, H, T, seed, 1.0)
+    k8, sk = _codes(orc, B, H, N, seed + 1, 1.0)
+    v8, sv = _codes(orc, B, H, N, seed + 2, 1.0)
+    sq = (sq * np.float32(qscale)).astype(np.float32)  # moderate logits
+    return q8, k8, v8, sq, sk, sv
+
+
+def _naive(orc, q8, k8, v8, sq, sk, sv):
+    q = orc.e4m3_decode(q8) * sq[..., None, None]
+    k = orc.e4m3_decode(k8) * sk[..., None, None]
+    v = orc.e4m3_decode(v8) * sv[..., None, None]
+    x = np.einsum("bhtd,bhnd->bhtn", q, k) / 8.0
+    x -= x.max(-1, keepdims=True)
+    p = np.exp(x)
+    o = np.einsum("bhtn,bhnd->bhtd", p, v) / p.sum(-1)[..., None]
+    return o.transpose(0, 2, 1, 3)  # [B,T,H,d]
+
+
+@pytest.mark.parametrize("bc", [1, 7, 128, 300])
+def test_unquantised_p_matches_naive_softmax(orc, bc):
+    q8, k8, v8, sq, sk, sv = _problem(orc)
+    _, out, _ = orc.attention(q8, k8, v8, sq, sk, sv, bc=bc, quant_p=False)
+    ref = _naive(orc, q8, k8, v8, sq, sk, sv)
+    assert np.abs(out - ref).max() <= 1e-5 * np.abs(ref).max() + 1e-7
+
+
+def test_exact_reference_matches_naive(orc):
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((2, 9, 3, 64)).astype(np.float16)
+    k = rng.standard_normal((2, 20, 3, 64)).astype(np.float16)
+    v = rng.standard_normal((2, 20, 3, 64)).astype(np.float16)
+    got = orc.attention_exact(q, k, v)
+    qd, kd, vd = (a.astype(np.float64).transpose(0, 2, 1, 3) for a in (q, k, v))
+    x = qd @ kd.transpose(0, 1, 3, 2) / 8.0
+    p = np.exp(x - x.max(-1, keepdims=True))
+    want = ((p @ vd) / p.sum(-1)[..., None]).transpose(0, 2, 1, 3)
+    assert np.abs(got - want).max() < 1e-12
+
+
+def test_golden_worked_example(orc):
+    lines = {ln.split()[0]: ln.split()[1:] for ln in open(os.path.join(GOLDEN, "softmax_worked_example.txt"))
+             if ln.strip() and ln[0] != "#"}
+    k2 = np.float32(LOG2E / 8.0)
+    sk = np.float32(1.0) / k2
+    for cand in (sk, np.nextafter(sk, np.float32(0)), np.nextafter(sk, np.float32(1e9))):
+        if np.float32(np.float32(1.0) * cand) * k2 == np.float32(1.0):
+            sk = cand
+            break
+    assert np.float32(sk * k2) == np.float32(1.0)
+    q8 = np.full((1, 1, 1, 64), 0x38, np.uint8)
+    k8 = np.stack([np.full(64, c, np.uint8) for c in (0x00, 0x08, 0x10)])[None, None]
+    v8 = np.stack([np.full(64, c, np.uint8) for c in (0x38, 0x40, 0x48)])[None, None]
+    one = np.ones((1, 1), np.float32)
+    for bc in (1, 2, 128):
+        o16, o, _ = orc.attention(q8, k8, v8, one, np.full((1, 1), sk, np.float32), one, bc=bc)
+        assert (o == float(lines["out"][0])).all(), (bc, o[0, 0, 0, :4])
+        assert (o16.astype(np.float64) == 3.0).all()
+
+
+@pytest.mark.parametrize("bc", [7, 128])
+def test_zero_query_gives_mean_of_v(orc, bc):
+    _, k8, v8, sq, sk, sv = _problem(orc)
+    q8 = np.zeros((1, 2, 5, 64), np.uint8)
+    o16, o, _ = orc.attention(q8, k8, v8, sq, sk, sv, bc=bc)
+    mean = orc.e4m3_decode(v8).mean(axis=2) * sv[..., None]      # [B,H,d]
+    assert np.allclose(o, mean[:, None, :, :], rtol=1e-12, atol=1e-15)
+    assert (o16.view(np.uint16) == orc.f16_encode(np.broadcast_to(mean[:, None], o.shape))).all()
+
+
+def test_constant_v_normalises_to_one(orc):
+    q8, k8, _, sq, sk, _ = _problem(orc)
+    v8 = np.full_like(k8, 0x38)
+    sv = np.ones_like(sq)
+    o16, o, _ = orc.attention(q8, k8, v8, sq, sk, sv, bc=16)
+    assert np.abs(o - 1.0).max() < 1e-14
+    assert (o16.astype(np.float64) == 1.0).all()
+
+
+def test_materialised_p_matches_online(orc):
+    """Full P matrix in numpy (fp32 logits in e order, torch e4m3 cast) vs the online oracle with one tile."""
+    q8, k8, v8, sq, sk, sv = _problem(orc, T=24, N=200, seed=7, qscale=1.0)
+    qf = orc.e4m3_decode(q8).astype(np.float32)
+    kf = orc.e4m3_decode(k8).astype(np.float32)
+    z = np.zeros((1, 2, 24, 200), np.float32)
+    for e in range(64):
+        z = (z + qf[..., e:e + 1] * kf[..., e][:, :, None, :]).astype(np.float32)
+    c2 = (np.float32(sq * sk) * np.float32(LOG2E / 8.0)).astype(np.float32)[..., None, None]
+    m2 = (z.max(-1, keepdims=True) * c2).astype(np.float32)
+    t = (z.astype(np.float64) * c2.astype(np.float64) - m2.astype(np.float64)).astype(np.float32)
+    p = np.exp2(t.astype(np.float64)).astype(np.float32)
+    p8 = orc.e4m3_decode(torch.from_numpy(p).to(torch.float8_e4m3fn).view(torch.uint8).numpy())
+    vf = orc.e4m3_decode(v8)
+    want = (np.einsum("bhtn,bhnd->bhtd", p8, vf) / p8.sum(-1)[..., None] * sv[..., None, None]).transpose(0, 2, 1, 3)
+    _, out, allow = orc.attention(q8, k8, v8, sq, sk, sv, bc=200, delta=1e-6)
+    assert (np.abs(out - want) <= 1e-12 + allow).all()
+
+
+def test_context_permutation(orc):
+    q8, k8, v8, sq, sk, sv = _problem(orc, N=256, seed=11)
+    perm = np.random.default_rng(0).permutation(256)
+    _, o1, _ = orc.attention(q8, k8, v8, sq, sk, sv, bc=256)
+    _, o2, _ = orc.attention(q8, k8[:, :, perm], v8[:, :, perm], sq, sk, sv, bc=256)
+    assert np.abs(o1 - o2).max() <= 1e-12 * np.abs(o1).max()
+    # with several tiles each tile quantises P against its own running max, so a
+    # permutation moves outputs by the e4m3 quantisation noise of P only
+    _, o3, _ = orc.attention(q8, k8[:, :, perm], v8[:, :, perm], sq, sk, sv, bc=16)
+    assert np.abs(o1 - o3).mean() < 3e-3 and np.abs(o1 - o3).max() < 5e-2
+
+
+def test_cached_split_is_partition_invariant(orc):
+    q8, k8, v8, sq, sk, sv = _problem(orc, T=33, N=700, seed=13)
+    full16, full, _ = orc.attention(q8, k8, v8, sq, sk, sv, split=256)
+    for part in (1, 5, 16):
+        for r0 in range(0, 33, part):
+            rows = np.arange(r0, min(33, r0 + part))
+            o16, o, _ = orc.attention(q8, k8, v8, sq, sk, sv, rows=rows, split=256)
+            assert (o == full[:, rows]).all()
+            assert (o16.view(np.uint16) == full16[:, rows].view(np.uint16)).all()
+
+
+def test_split_covering_all_keys_equals_one_pass(orc):
+    q8, k8, v8, sq, sk, sv = _problem(orc, T=20, N=300, seed=17)
+    a16, a, _ = orc.attention(q8, k8, v8, sq, sk, sv, split=0)
+    b16, b, _ = orc.attention(q8, k8, v8, sq, sk, sv, split=512)
+    assert (a == b).all() and (a16.view(np.uint16) == b16.view(np.uint16)).all()
+    _, c, _ = orc.attention(q8, k8, v8, sq, sk, sv, split=128)
+    assert np.abs(a - c).mean() < 3e-3 and np.abs(a - c).max() < 5e-2
+
+
+def test_allowance_properties(orc):
+    q8, k8, v8, sq, sk, sv = _problem(orc, seed=19)
+    _, _, a0 = orc.attention(q8, k8, v8, sq, sk, sv, delta=0.0)
+    _, _, a1 = orc.attention(q8, k8, v8, sq, sk, sv, delta=1e-4)
+    _, _, a2 = orc.attention(q8, k8, v8, sq, sk, sv, delta=1e-2)
+    assert (a0 == 0).all() and (a1 >= 0).all() and (a2 >= a1).all() and a2.max() > 0
+
+
+def test_lossless_when_inputs_are_e4m3_values(orc):
+    """Inputs that are exactly e4m3 values times 2^-6 quantise losslessly, so with P
+    unquantised the scales -> codes -> attention chain equals exact attention."""
+    rng = np.random.default_rng(23)
+    def exact_e4m3_tensor(rows):
+        c = rng.integers(0, 0x7E, size=(1, rows, 2, 64)).astype(np.uint8) | (rng.integers(0, 2, (1, rows, 2, 64)) << 7).astype(np.uint8)
+        c[0, 0, :, 0] = 0x7E  # every head reaches 448 -> scale exactly 2^-6
+        return (orc.e4m3_decode(c) * 2.0 ** -6).astype(np.float16)
+    q, k, v = exact_e4m3_tensor(50), exact_e4m3_tensor(300), exact_e4m3_tensor(300)
+    q = (q.astype(np.float32) * np.float32(0.125)).astype(np.float16)   # exact: power of two
+    sq, sk, sv = (orc.context_scales(x, x.shape[1]) for x in (q, k, v))
+    assert (sk == 2.0 ** -6).all() and (sv == 2.0 ** -6).all() and (sq == 2.0 ** -9).all()
+    q8, k8, v8 = orc.quantize(q, sq), orc.quantize(k, sk), orc.quantize(v, sv)
+    assert (orc.e4m3_decode(q8).transpose(0, 2, 1, 3) * 2.0 ** -9 == q.astype(np.float64)).all()
+    _, out, _ = orc.attention(q8, k8, v8, sq, sk, sv, quant_p=False)
+    exact = orc.attention_exact(q, k, v)
+    assert np.abs(out - exact).max() <= 1e-5 * np.abs(exact).max()
