@@ -1,0 +1,250 @@
+"""ctypes binding of ``libsdm_fp8.so`` (the C ABI in ``include/sdm_fp8.h``).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  torch supplies device memory, the current stream and dtype checks.
+If the shared library is missing, every call raises -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsdm_fp8.so")
+
+SDM_OK = 0
+STATUS_NAMES = {0: "SDM_OK", 1: "SDM_ERR_INVALID_ARG", 2: "SDM_ERR_UNSUPPORTED", 3: "SDM_ERR_WORKSPACE",
+                4: "SDM_ERR_DEVICE_MISMATCH", 5: "SDM_ERR_CACHE_MISMATCH", 6: "SDM_ERR_TIMEOUT",
+                7: "SDM_ERR_CUDA"}
+OP_QUANTIZE_CONTEXT, OP_ICL_ATTENTION, OP_CACHED_ATTENTION = 0, 1, 2
+KV_TILE = 128
+SPLIT_KEYS = 16384
+HEAD_DIM = 64
+
+# Every symbol the header declares (checked by the ABI tests).
+EXPORTS = ("sdm_status_string", "sdm_version", "sdm_cache_layout", "sdm_workspace_size", "sdm_qscale_fused",
+           "sdm_fp8_quantize_context", "sdm_fp8_attention", "sdm_icl_attention", "sdm_cached_attention",
+           "sdm_sync_status")
+
+
+class SdmError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} ({_status_string(status)})")
+
+
+class CacheStruct(ctypes.Structure):
+    _fields_ = [("k8", ctypes.c_void_p), ("v8t", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("n_ctx", ctypes.c_int64), ("ld_v", ctypes.c_int64), ("batch", ctypes.c_int32),
+                ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("device", ctypes.c_int32),
+                ("filled", ctypes.c_int32)]
+
+
+_lib = None
+_P, _I32, _I64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsdm_fp8.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run fp8_quant_logscale_b200/build.py "
+                               "(or __graft_entry__.build()) first; there is no CPU fallback")
+        L = ctypes.CDLL(LIB_PATH)
+        L.sdm_status_string.restype = ctypes.c_char_p
+        L.sdm_status_string.argtypes = [ctypes.c_int]
+        L.sdm_version.restype = _I32
+        L.sdm_version.argtypes = []
+        L.sdm_cache_layout.restype = ctypes.c_int
+        L.sdm_cache_layout.argtypes = [_I32, _I64, _I32, _I32, ctypes.POINTER(_SZ), ctypes.POINTER(_SZ),
+                                       ctypes.POINTER(_SZ), ctypes.POINTER(_I64)]
+        L.sdm_workspace_size.restype = _SZ
+        L.sdm_workspace_size.argtypes = [ctypes.c_int, _I32, _I64, _I64, _I32, _I32, _I32]
+        L.sdm_qscale_fused.restype = ctypes.c_int
+        L.sdm_qscale_fused.argtypes = [_P, _P, _I32, _I64, _I32, _I32, _I64, _P, _P, _P]
+        L.sdm_fp8_quantize_context.restype = ctypes.c_int
+        L.sdm_fp8_quantize_context.argtypes = [_P, _P, _P, _I32, _I64, _I64, _I32, _I32, _P,
+                                               ctypes.POINTER(CacheStruct), _P, _SZ, _P]
+        L.sdm_fp8_attention.restype = ctypes.c_int
+        L.sdm_fp8_attention.argtypes = [_P, _I32, _I64, ctypes.POINTER(CacheStruct), _P, _I32, _P, _SZ, _P]
+        L.sdm_icl_attention.restype = ctypes.c_int
+        L.sdm_icl_attention.argtypes = [_P, _P, _P, _I32, _I64, _I64, _I32, _I32, _P, _P, _P,
+                                        ctypes.POINTER(CacheStruct), _P, _SZ, _P]
+        L.sdm_cached_attention.restype = ctypes.c_int
+        L.sdm_cached_attention.argtypes = [_P, _I32, _I64, _I32, _I32, ctypes.POINTER(CacheStruct), _P, _P, _P,
+                                           _P, _SZ, _P]
+        L.sdm_sync_status.restype = ctypes.c_int
+        L.sdm_sync_status.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_uint32)]
+        _lib = L
+    return _lib
+
+
+def _status_string(status: int) -> str:
+    try:
+        return lib().sdm_status_string(int(status)).decode()
+    except Exception:  # pragma: no cover - only while reporting another error
+        return "?"
+
+
+def _check(status: int, what: str) -> None:
+    if status != SDM_OK:
+        raise SdmError(status, what)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _want(t: torch.Tensor, dtype: torch.dtype, name: str, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-d tensor")
+
+
+# ------------------------------------------------------------------- sizes
+
+def workspace_size(op: int, batch: int, n_ctx: int, n_query: int, heads: int, keep_cache: bool = True) -> int:
+    return int(lib().sdm_workspace_size(op, batch, n_ctx, n_query, heads, HEAD_DIM, 1 if keep_cache else 0))
+
+
+def new_workspace(nbytes: int, device) -> torch.Tensor:
+    """Zero-filled workspace (the error word must start at zero)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def sync_status(ws: torch.Tensor) -> tuple[int, int]:
+    """(status, raw error flags) of the kernels that used `ws`; synchronises the current stream."""
+    flags = ctypes.c_uint32(0)
+    st = lib().sdm_sync_status(_ptr(ws), _stream(ws.device), ctypes.byref(flags))
+    return int(st), int(flags.value)
+
+
+class FP8Cache:
+    """Caller-owned FP8 K/V cache (k8 [B,H,N,64], v8t [B,H,64,ld_v], scales [3,B,H])."""
+
+    def __init__(self, batch: int, n_ctx: int, heads: int, device):
+        kb, vb, sb, ld = _SZ(), _SZ(), _SZ(), _I64()
+        _check(lib().sdm_cache_layout(batch, n_ctx, heads, HEAD_DIM, ctypes.byref(kb), ctypes.byref(vb),
+                                      ctypes.byref(sb), ctypes.byref(ld)), "sdm_cache_layout")
+        device = torch.device(device)
+        self.k8 = torch.empty((batch, heads, n_ctx, HEAD_DIM), dtype=torch.uint8, device=device)
+        self.v8t = torch.empty((batch, heads, HEAD_DIM, ld.value), dtype=torch.uint8, device=device)
+        self.scales = torch.empty((3, batch, heads), dtype=torch.float32, device=device)
+        assert self.k8.numel() == kb.value and self.v8t.numel() == vb.value and self.scales.numel() * 4 == sb.value
+        self.struct = CacheStruct(self.k8.data_ptr(), self.v8t.data_ptr(), self.scales.data_ptr(), n_ctx, ld.value,
+                                  batch, heads, HEAD_DIM, device.index if device.index is not None else 0, 0)
+
+    @property
+    def filled(self) -> bool:
+        return self.struct.filled == 1
+
+    @property
+    def n_ctx(self) -> int:
+        return int(self.struct.n_ctx)
+
+    @property
+    def ld_v(self) -> int:
+        return int(self.struct.ld_v)
+
+
+# ------------------------------------------------------------- operations
+
+def qscale_fused(q: torch.Tensor, c_h: torch.Tensor, n_len: int, gate: torch.Tensor | None = None,
+                 out: torch.Tensor | None = None) -> torch.Tensor:
+    """LogScale / GatedLogScale of q [B, rows, H, 64] fp16 with shared key length n_len."""
+    _want(q, torch.float16, "q", 4)
+    B, rows, H, d = q.shape
+    _want(c_h, torch.float32, "c_h", 1)
+    if gate is not None:
+        _want(gate, torch.float16, "gate", 3)
+    out = torch.empty_like(q) if out is None else out
+    with torch.cuda.device(q.device):
+        _check(lib().sdm_qscale_fused(_ptr(q), _ptr(out), B, rows, H, d, int(n_len), _ptr(c_h), _ptr(gate),
+                                      _stream(q.device)), "sdm_qscale_fused")
+    return out
+
+
+def fp8_quantize_context(q_scaled: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_ctx: int,
+                         cache: FP8Cache | None = None, ws: torch.Tensor | None = None):
+    """Context-scale e4m3 quantisation.  Returns (q8 [B,H,T,64] uint8, cache)."""
+    _want(q_scaled, torch.float16, "q_scaled", 4)
+    _want(k, torch.float16, "k", 4)
+    _want(v, torch.float16, "v", 4)
+    B, T, H, d = q_scaled.shape
+    M = T - n_ctx
+    dev = q_scaled.device
+    cache = FP8Cache(B, n_ctx, H, dev) if cache is None else cache
+    q8 = torch.empty((B, H, T, d), dtype=torch.uint8, device=dev)
+    need = workspace_size(OP_QUANTIZE_CONTEXT, B, n_ctx, M, H)
+    ws = new_workspace(need, dev) if ws is None else ws
+    with torch.cuda.device(dev):
+        _check(lib().sdm_fp8_quantize_context(_ptr(q_scaled), _ptr(k), _ptr(v), B, n_ctx, M, H, d, _ptr(q8),
+                                              ctypes.byref(cache.struct), _ptr(ws), ws.numel(), _stream(dev)),
+               "sdm_fp8_quantize_context")
+    return q8, cache
+
+
+def fp8_attention(q8: torch.Tensor, cache: FP8Cache, split: bool = False, out: torch.Tensor | None = None,
+                  ws: torch.Tensor | None = None) -> torch.Tensor:
+    """Step 3 alone on quantised rows q8 [B,H,rows,64].  Returns out [B,rows,H,64] fp16."""
+    _want(q8, torch.uint8, "q8", 4)
+    B, H, rows, d = q8.shape
+    dev = q8.device
+    out = torch.empty((B, rows, H, d), dtype=torch.float16, device=dev) if out is None else out
+    need = workspace_size(OP_CACHED_ATTENTION, B, cache.n_ctx, rows, H)
+    ws = new_workspace(need, dev) if ws is None else ws
+    with torch.cuda.device(dev):
+        _check(lib().sdm_fp8_attention(_ptr(q8), B, rows, ctypes.byref(cache.struct), _ptr(out), 1 if split else 0,
+                                       _ptr(ws), ws.numel(), _stream(dev)), "sdm_fp8_attention")
+    return out
+
+
+def icl_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_ctx: int, c_h: torch.Tensor,
+                  gate: torch.Tensor | None = None, cache: FP8Cache | None = None, out: torch.Tensor | None = None,
+                  ws: torch.Tensor | None = None) -> torch.Tensor:
+    """One call of the layer: q [B,T,H,64] raw fp16, k/v [B,N,H,64] fp16 -> out [B,T,H,64] fp16."""
+    _want(q, torch.float16, "q", 4)
+    _want(k, torch.float16, "k", 4)
+    _want(v, torch.float16, "v", 4)
+    _want(c_h, torch.float32, "c_h", 1)
+    if gate is not None:
+        _want(gate, torch.float16, "gate", 3)
+    B, T, H, d = q.shape
+    M = T - n_ctx
+    dev = q.device
+    out = torch.empty_like(q) if out is None else out
+    need = workspace_size(OP_ICL_ATTENTION, B, n_ctx, M, H, keep_cache=cache is not None)
+    ws = new_workspace(need, dev) if ws is None else ws
+    with torch.cuda.device(dev):
+        _check(lib().sdm_icl_attention(_ptr(q), _ptr(k), _ptr(v), B, n_ctx, M, H, d, _ptr(c_h), _ptr(gate),
+                                       _ptr(out), None if cache is None else ctypes.byref(cache.struct), _ptr(ws),
+                                       ws.numel(), _stream(dev)), "sdm_icl_attention")
+    return out
+
+
+def cached_attention(q: torch.Tensor, cache: FP8Cache, c_h: torch.Tensor, gate: torch.Tensor | None = None,
+                     out: torch.Tensor | None = None, ws: torch.Tensor | None = None) -> torch.Tensor:
+    """Cached prediction: q [B,M,H,64] raw fp16 against a filled cache -> out [B,M,H,64] fp16."""
+    _want(q, torch.float16, "q", 4)
+    _want(c_h, torch.float32, "c_h", 1)
+    if gate is not None:
+        _want(gate, torch.float16, "gate", 3)
+    B, M, H, d = q.shape
+    dev = q.device
+    out = torch.empty_like(q) if out is None else out
+    need = workspace_size(OP_CACHED_ATTENTION, B, cache.n_ctx, M, H)
+    ws = new_workspace(need, dev) if ws is None else ws
+    with torch.cuda.device(dev):
+        _check(lib().sdm_cached_attention(_ptr(q), B, M, H, d, ctypes.byref(cache.struct), _ptr(c_h), _ptr(gate),
+                                          _ptr(out), _ptr(ws), ws.numel(), _stream(dev)), "sdm_cached_attention")
+    return out

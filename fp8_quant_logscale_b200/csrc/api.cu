@@ -1,0 +1,413 @@
+// api.cu -- the C ABI declared in include/sdm_fp8.h: argument validation,
+// workspace carving, and the launch sequences of the four layer operations.
+// Every argument error is reported before any work is enqueued; nothing here
+// allocates device memory.
+#include <math.h>
+#include <string.h>
+
+#include "../../include/sdm_fp8.h"
+#include "kernels.cuh"
+
+using namespace sdm;
+
+namespace {
+
+constexpr size_t kAlign = 1024;
+constexpr size_t kErrBytes = 256;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  return dev;
+}
+
+// True if p is device (or managed) memory on device `dev`.
+bool on_device(const void* p, int dev) {
+  if (p == nullptr) return false;
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) && at.device == dev;
+}
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+sdm_status check_shape(int32_t B, int64_t rows_a, int64_t rows_b, int32_t H, int32_t d) {
+  if (B < 1 || H < 1 || rows_a < 0 || rows_b < 0) return SDM_ERR_INVALID_ARG;
+  if (d != kHeadDim) return SDM_ERR_UNSUPPORTED;
+  if (H > 128) return SDM_ERR_UNSUPPORTED;
+  // TMA coordinates and grid sizes are 32-bit: keep every row count and B*H in range
+  if (rows_a > (int64_t)1 << 30 || rows_b > (int64_t)1 << 30 || (int64_t)B * H > 65535) return SDM_ERR_UNSUPPORTED;
+  return SDM_OK;
+}
+
+// Checks a tensor pointer: non-null, 16-byte aligned, device memory of `dev`.
+sdm_status check_tensor(const void* p, int dev) {
+  if (p == nullptr || !aligned(p, 16)) return SDM_ERR_INVALID_ARG;
+  if (!on_device(p, dev)) return SDM_ERR_DEVICE_MISMATCH;
+  return SDM_OK;
+}
+
+#define SDM_TRY(expr)                       \
+  do {                                      \
+    const sdm_status _st = (expr);          \
+    if (_st != SDM_OK) return _st;          \
+  } while (0)
+
+#define SDM_CUDA(expr)                      \
+  do {                                      \
+    if ((expr) != cudaSuccess) {            \
+      cudaGetLastError();                   \
+      return SDM_ERR_CUDA;                  \
+    }                                       \
+  } while (0)
+
+// Workspace carve-up.  Offsets are 1 KB aligned; the error word sits at 0.
+struct WsLayout {
+  size_t amax = 0, q8 = 0, k8 = 0, v8t = 0, scales = 0, part_acc = 0, part_ml = 0, total = 0;
+};
+
+int64_t n_splits_for(int64_t n_ctx) { return (n_ctx + kSplitKeys - 1) / kSplitKeys; }
+
+WsLayout ws_layout(sdm_op op, int32_t B, int64_t N, int64_t M, int32_t H, int32_t keep_cache) {
+  WsLayout w;
+  const size_t BH = (size_t)B * H;
+  size_t off = kErrBytes;
+  w.amax = off;
+  off = align_up(off + 3 * BH * sizeof(uint32_t), kAlign);
+  if (op == SDM_OP_QUANTIZE_CONTEXT) {
+    w.total = off;
+    return w;
+  }
+  const int64_t rows = (op == SDM_OP_ICL_ATTENTION) ? N + M : M;
+  w.q8 = off;
+  off = align_up(off + BH * (size_t)rows * kHeadDim, kAlign);
+  if (op == SDM_OP_ICL_ATTENTION && !keep_cache) {
+    const int64_t ld = round_up(N, kKvTile);
+    w.k8 = off;
+    off = align_up(off + BH * (size_t)N * kHeadDim, kAlign);
+    w.v8t = off;
+    off = align_up(off + BH * kHeadDim * (size_t)ld, kAlign);
+    w.scales = off;
+    off = align_up(off + 3 * BH * sizeof(float), kAlign);
+  }
+  if (op == SDM_OP_CACHED_ATTENTION) {
+    const size_t S = (size_t)n_splits_for(N);
+    w.part_acc = off;
+    off = align_up(off + S * BH * (size_t)M * kHeadDim * sizeof(float), kAlign);
+    w.part_ml = off;
+    off = align_up(off + S * BH * (size_t)M * 2 * sizeof(float), kAlign);
+  }
+  w.total = off;
+  return w;
+}
+
+sdm_status check_ws(void* ws, size_t ws_bytes, size_t need, int dev) {
+  if (ws == nullptr || ws_bytes < need) return SDM_ERR_WORKSPACE;
+  if (!aligned(ws, 256)) return SDM_ERR_INVALID_ARG;
+  if (!on_device(ws, dev)) return SDM_ERR_DEVICE_MISMATCH;
+  return SDM_OK;
+}
+
+// Validates the cache descriptor against a call's B/H/d and the device.
+sdm_status check_cache(const sdm_fp8_cache* c, int32_t B, int32_t H, int32_t d, int dev, bool need_filled) {
+  if (c == nullptr) return SDM_ERR_INVALID_ARG;
+  if (c->batch != B || c->heads != H || c->head_dim != d || c->device != dev || c->n_ctx < 1 ||
+      c->ld_v != round_up(c->n_ctx, kKvTile))
+    return SDM_ERR_CACHE_MISMATCH;
+  if (need_filled && c->filled != 1) return SDM_ERR_CACHE_MISMATCH;
+  if (c->k8 == nullptr || c->v8t == nullptr || c->scales == nullptr) return SDM_ERR_INVALID_ARG;
+  if (!aligned(c->k8, 16) || !aligned(c->v8t, 16) || !aligned(c->scales, 16)) return SDM_ERR_INVALID_ARG;
+  if (!on_device(c->k8, dev) || !on_device(c->v8t, dev) || !on_device(c->scales, dev))
+    return SDM_ERR_CACHE_MISMATCH;
+  return SDM_OK;
+}
+
+QScale make_qscale(int64_t n_len, const float* c_h, const void* gate) {
+  QScale qs;
+  qs.enabled = true;
+  // fp32 natural log of the shared integer length, clamped at 1, on the host
+  qs.lam = logf(static_cast<float>(n_len < 1 ? 1 : n_len));
+  qs.c_h = c_h;
+  qs.gate = reinterpret_cast<const __half*>(gate);
+  return qs;
+}
+
+QScale no_qscale() {
+  QScale qs;
+  qs.enabled = false;
+  qs.lam = 0.0f;
+  qs.c_h = nullptr;
+  qs.gate = nullptr;
+  return qs;
+}
+
+// amax -> scales -> Q8 / K8 / V8^T.  `qs` is applied to Q (enabled: raw q in).
+sdm_status run_quantize(const __half* q, const __half* k, const __half* v, int32_t B, int64_t N, int64_t M,
+                        int32_t H, QScale qs, uint8_t* q8, uint8_t* k8, uint8_t* v8t, int64_t ld, float* scales,
+                        uint8_t* ws_base, const WsLayout& w, cudaStream_t st) {
+  const int64_t T = N + M;
+  uint32_t* amax = reinterpret_cast<uint32_t*>(ws_base + w.amax);
+  SDM_CUDA(cudaMemsetAsync(amax, 0, 3 * (size_t)B * H * sizeof(uint32_t), st));
+  RowsDesc dq{q, B, H, T}, dk{k, B, H, N}, dv{v, B, H, N};
+  SDM_CUDA(launch_context_amax(dq, qs, dk, dv, N, amax, st));
+  SDM_CUDA(launch_scales_from_amax(amax, B * H, scales, st));
+  const int64_t BH = (int64_t)B * H;
+  SDM_CUDA(launch_quantize_rows(dq, qs, T, scales, q8, T, st));
+  SDM_CUDA(launch_quantize_rows(dk, no_qscale(), N, scales + BH, k8, N, st));
+  SDM_CUDA(launch_quantize_vt(dv, N, scales + 2 * BH, v8t, ld, st));
+  return SDM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sdm_status_string(sdm_status s) {
+  switch (s) {
+    case SDM_OK: return "SDM_OK";
+    case SDM_ERR_INVALID_ARG: return "SDM_ERR_INVALID_ARG: null, misaligned or out-of-range argument";
+    case SDM_ERR_UNSUPPORTED: return "SDM_ERR_UNSUPPORTED: head_dim must be 64, heads 1..128, rows <= 2^30";
+    case SDM_ERR_WORKSPACE: return "SDM_ERR_WORKSPACE: workspace missing or too small";
+    case SDM_ERR_DEVICE_MISMATCH: return "SDM_ERR_DEVICE_MISMATCH: pointer is not device memory of the current device";
+    case SDM_ERR_CACHE_MISMATCH: return "SDM_ERR_CACHE_MISMATCH: FP8 cache shape, device or state disagrees with the call";
+    case SDM_ERR_TIMEOUT: return "SDM_ERR_TIMEOUT: an in-kernel bounded wait gave up";
+    case SDM_ERR_CUDA: return "SDM_ERR_CUDA: a CUDA runtime call or kernel launch failed";
+  }
+  return "SDM_ERR_UNKNOWN";
+}
+
+int32_t sdm_version(void) { return 100; }
+
+sdm_status sdm_cache_layout(int32_t B, int64_t N, int32_t H, int32_t d, size_t* k8_bytes, size_t* v8t_bytes,
+                            size_t* scales_bytes, int64_t* ld_v) {
+  SDM_TRY(check_shape(B, N, 0, H, d));
+  if (N < 1) return SDM_ERR_INVALID_ARG;
+  const int64_t ld = round_up(N, kKvTile);
+  if (k8_bytes) *k8_bytes = (size_t)B * H * N * kHeadDim;
+  if (v8t_bytes) *v8t_bytes = (size_t)B * H * kHeadDim * ld;
+  if (scales_bytes) *scales_bytes = 3 * (size_t)B * H * sizeof(float);
+  if (ld_v) *ld_v = ld;
+  return SDM_OK;
+}
+
+size_t sdm_workspace_size(sdm_op op, int32_t B, int64_t N, int64_t M, int32_t H, int32_t d, int32_t keep_cache) {
+  if (op != SDM_OP_QUANTIZE_CONTEXT && op != SDM_OP_ICL_ATTENTION && op != SDM_OP_CACHED_ATTENTION) return 0;
+  if (check_shape(B, N, M, H, d) != SDM_OK || N < 1) return 0;
+  return ws_layout(op, B, N, M, H, keep_cache).total;
+}
+
+sdm_status sdm_qscale_fused(const void* q, void* q_out, int32_t B, int64_t rows, int32_t H, int32_t d,
+                            int64_t n_len, const float* c_h, const void* gate, void* stream) {
+  SDM_TRY(check_shape(B, rows, 0, H, d));
+  if (n_len < 1) return SDM_ERR_INVALID_ARG;
+  const int dev = current_device();
+  if (dev < 0) return SDM_ERR_CUDA;
+  SDM_TRY(check_tensor(q, dev));
+  SDM_TRY(check_tensor(q_out, dev));
+  if (c_h == nullptr || !aligned(c_h, 4)) return SDM_ERR_INVALID_ARG;
+  if (!on_device(c_h, dev)) return SDM_ERR_DEVICE_MISMATCH;
+  if (gate != nullptr) {
+    if (!aligned(gate, 2)) return SDM_ERR_INVALID_ARG;
+    if (!on_device(gate, dev)) return SDM_ERR_DEVICE_MISMATCH;
+  }
+  if (rows == 0) return SDM_OK;
+  SDM_CUDA(launch_qscale(reinterpret_cast<const __half*>(q), reinterpret_cast<__half*>(q_out), B, rows, H,
+                         make_qscale(n_len, c_h, gate), as_stream(stream)));
+  return SDM_OK;
+}
+
+sdm_status sdm_fp8_quantize_context(const void* q_scaled, const void* k, const void* v, int32_t B, int64_t N,
+                                    int64_t M, int32_t H, int32_t d, uint8_t* q8, sdm_fp8_cache* cache, void* ws,
+                                    size_t ws_bytes, void* stream) {
+  SDM_TRY(check_shape(B, N, M, H, d));
+  if (N < 1) return SDM_ERR_INVALID_ARG;
+  const int dev = current_device();
+  if (dev < 0) return SDM_ERR_CUDA;
+  SDM_TRY(check_tensor(q_scaled, dev));
+  SDM_TRY(check_tensor(k, dev));
+  SDM_TRY(check_tensor(v, dev));
+  SDM_TRY(check_tensor(q8, dev));
+  SDM_TRY(check_cache(cache, B, H, d, dev, false));
+  if (cache->n_ctx != N) return SDM_ERR_CACHE_MISMATCH;
+  const WsLayout w = ws_layout(SDM_OP_QUANTIZE_CONTEXT, B, N, M, H, 1);
+  SDM_TRY(check_ws(ws, ws_bytes, w.total, dev));
+  cudaStream_t st = as_stream(stream);
+  SDM_TRY(run_quantize(reinterpret_cast<const __half*>(q_scaled), reinterpret_cast<const __half*>(k),
+                       reinterpret_cast<const __half*>(v), B, N, M, H, no_qscale(), q8, cache->k8, cache->v8t,
+                       cache->ld_v, cache->scales, reinterpret_cast<uint8_t*>(ws), w, st));
+  cache->filled = 1;
+  return SDM_OK;
+}
+
+sdm_status sdm_fp8_attention(const uint8_t* q8, int32_t B, int64_t rows, const sdm_fp8_cache* cache, void* out,
+                             int32_t split, void* ws, size_t ws_bytes, void* stream) {
+  if (cache == nullptr) return SDM_ERR_INVALID_ARG;
+  SDM_TRY(check_shape(B, cache->n_ctx, rows, cache->heads, cache->head_dim));
+  if (split != 0 && split != 1) return SDM_ERR_INVALID_ARG;
+  const int dev = current_device();
+  if (dev < 0) return SDM_ERR_CUDA;
+  SDM_TRY(check_cache(cache, B, cache->heads, cache->head_dim, dev, true));
+  if (rows == 0) return SDM_OK;
+  SDM_TRY(check_tensor(q8, dev));
+  SDM_TRY(check_tensor(out, dev));
+  const int32_t H = cache->heads;
+  const WsLayout w = ws_layout(SDM_OP_CACHED_ATTENTION, B, cache->n_ctx, rows, H, 1);
+  SDM_TRY(check_ws(ws, ws_bytes, split ? w.total : kErrBytes, dev));
+  cudaStream_t st = as_stream(stream);
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  AttnArgs a;
+  a.B = B;
+  a.H = H;
+  a.T = rows;
+  a.N = cache->n_ctx;
+  a.ld_v = cache->ld_v;
+  a.scales = cache->scales;
+  a.n_splits = split ? n_splits_for(cache->n_ctx) : 1;
+  a.split_keys = kSplitKeys;
+  a.out = reinterpret_cast<__half*>(out);
+  a.part_acc = split ? reinterpret_cast<float*>(base + w.part_acc) : nullptr;
+  a.part_ml = split ? reinterpret_cast<float*>(base + w.part_ml) : nullptr;
+  a.err = reinterpret_cast<uint32_t*>(base);
+  SDM_CUDA(launch_attention(q8, cache->k8, cache->v8t, a, st));
+  if (split) SDM_CUDA(launch_splitkv_reduce(a, st));
+  return SDM_OK;
+}
+
+sdm_status sdm_icl_attention(const void* q, const void* k, const void* v, int32_t B, int64_t N, int64_t M,
+                             int32_t H, int32_t d, const float* c_h, const void* gate, void* out,
+                             sdm_fp8_cache* cache, void* ws, size_t ws_bytes, void* stream) {
+  SDM_TRY(check_shape(B, N, M, H, d));
+  if (N < 1) return SDM_ERR_INVALID_ARG;
+  const int dev = current_device();
+  if (dev < 0) return SDM_ERR_CUDA;
+  SDM_TRY(check_tensor(q, dev));
+  SDM_TRY(check_tensor(k, dev));
+  SDM_TRY(check_tensor(v, dev));
+  SDM_TRY(check_tensor(out, dev));
+  if (c_h == nullptr || !aligned(c_h, 4)) return SDM_ERR_INVALID_ARG;
+  if (!on_device(c_h, dev)) return SDM_ERR_DEVICE_MISMATCH;
+  if (gate != nullptr) {
+    if (!aligned(gate, 2)) return SDM_ERR_INVALID_ARG;
+    if (!on_device(gate, dev)) return SDM_ERR_DEVICE_MISMATCH;
+  }
+  if (cache != nullptr) {
+    SDM_TRY(check_cache(cache, B, H, d, dev, false));
+    if (cache->n_ctx != N) return SDM_ERR_CACHE_MISMATCH;
+  }
+  const WsLayout w = ws_layout(SDM_OP_ICL_ATTENTION, B, N, M, H, cache != nullptr);
+  SDM_TRY(check_ws(ws, ws_bytes, w.total, dev));
+  cudaStream_t st = as_stream(stream);
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  sdm_fp8_cache local;
+  sdm_fp8_cache* c = cache;
+  if (c == nullptr) {
+    memset(&local, 0, sizeof(local));
+    local.k8 = base + w.k8;
+    local.v8t = base + w.v8t;
+    local.scales = reinterpret_cast<float*>(base + w.scales);
+    local.n_ctx = N;
+    local.ld_v = round_up(N, kKvTile);
+    local.batch = B;
+    local.heads = H;
+    local.head_dim = d;
+    local.device = dev;
+    c = &local;
+  }
+  uint8_t* q8 = base + w.q8;
+  SDM_TRY(run_quantize(reinterpret_cast<const __half*>(q), reinterpret_cast<const __half*>(k),
+                       reinterpret_cast<const __half*>(v), B, N, M, H, make_qscale(N, c_h, gate), q8, c->k8, c->v8t,
+                       c->ld_v, c->scales, base, w, st));
+  c->filled = 1;
+  AttnArgs a;
+  a.B = B;
+  a.H = H;
+  a.T = N + M;
+  a.N = N;
+  a.ld_v = c->ld_v;
+  a.scales = c->scales;
+  a.n_splits = 1;
+  a.split_keys = kSplitKeys;
+  a.out = reinterpret_cast<__half*>(out);
+  a.part_acc = nullptr;
+  a.part_ml = nullptr;
+  a.err = reinterpret_cast<uint32_t*>(base);
+  SDM_CUDA(launch_attention(q8, c->k8, c->v8t, a, st));
+  return SDM_OK;
+}
+
+sdm_status sdm_cached_attention(const void* q, int32_t B, int64_t M, int32_t H, int32_t d,
+                                const sdm_fp8_cache* cache, const float* c_h, const void* gate, void* out, void* ws,
+                                size_t ws_bytes, void* stream) {
+  if (cache == nullptr) return SDM_ERR_INVALID_ARG;
+  SDM_TRY(check_shape(B, cache->n_ctx, M, H, d));
+  const int dev = current_device();
+  if (dev < 0) return SDM_ERR_CUDA;
+  SDM_TRY(check_cache(cache, B, H, d, dev, true));
+  if (c_h == nullptr || !aligned(c_h, 4)) return SDM_ERR_INVALID_ARG;
+  if (!on_device(c_h, dev)) return SDM_ERR_DEVICE_MISMATCH;
+  if (M == 0) return SDM_OK;
+  SDM_TRY(check_tensor(q, dev));
+  SDM_TRY(check_tensor(out, dev));
+  if (gate != nullptr) {
+    if (!aligned(gate, 2)) return SDM_ERR_INVALID_ARG;
+    if (!on_device(gate, dev)) return SDM_ERR_DEVICE_MISMATCH;
+  }
+  const int64_t N = cache->n_ctx;
+  const WsLayout w = ws_layout(SDM_OP_CACHED_ATTENTION, B, N, M, H, 1);
+  SDM_TRY(check_ws(ws, ws_bytes, w.total, dev));
+  cudaStream_t st = as_stream(stream);
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  uint8_t* q8 = base + w.q8;
+  // query scaling with the shared key length n = N, quantised with the context s_q
+  RowsDesc dq{reinterpret_cast<const __half*>(q), B, H, M};
+  SDM_CUDA(launch_quantize_rows(dq, make_qscale(N, c_h, gate), M, cache->scales, q8, M, st));
+  AttnArgs a;
+  a.B = B;
+  a.H = H;
+  a.T = M;
+  a.N = N;
+  a.ld_v = cache->ld_v;
+  a.scales = cache->scales;
+  a.n_splits = n_splits_for(N);
+  a.split_keys = kSplitKeys;
+  a.out = reinterpret_cast<__half*>(out);
+  a.part_acc = reinterpret_cast<float*>(base + w.part_acc);
+  a.part_ml = reinterpret_cast<float*>(base + w.part_ml);
+  a.err = reinterpret_cast<uint32_t*>(base);
+  SDM_CUDA(launch_attention(q8, cache->k8, cache->v8t, a, st));
+  SDM_CUDA(launch_splitkv_reduce(a, st));
+  return SDM_OK;
+}
+
+sdm_status sdm_sync_status(void* ws, void* stream, uint32_t* flags) {
+  if (ws == nullptr) return SDM_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaGetLastError();
+    return SDM_ERR_CUDA;
+  }
+  if (flags) *flags = word;
+  if (word != 0) {
+    if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess) {
+      cudaGetLastError();
+      return SDM_ERR_CUDA;
+    }
+    return SDM_ERR_TIMEOUT;
+  }
+  return SDM_OK;
+}
+
+}  // extern "C"

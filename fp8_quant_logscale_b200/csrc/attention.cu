@@ -1,0 +1,500 @@
+// attention.cu -- FP8 (e4m3) flash attention on the sm_100a tensor cores.
+//
+// Computes the in-context-learning attention of "[FP8 3/4] Integrate FP8
+// attention and caching into TabICLv2" (opening section): every row (context
+// or query) attends to all context keys, non-causal; probabilities are
+// quantised to e4m3 before the P.V product; the cached-prediction variant
+// ("model.predict(queries)" after "model.fit") splits the keys into
+// fixed-length chunks whose partial results a second kernel combines.
+//
+// One CTA owns two 128-row query tiles of one (batch, head) and streams the
+// keys of its range in 128-key tiles:
+//   warp 8      TMA producer: Q once, then K and V^T tiles into a 4-stage ring
+//               (separate "full" barriers for K and V, so S = Q K^T can start
+//               before V lands);
+//   warp 9      MMA issuer (one thread): S_t = Q_t K^T (tcgen05 kind::f8f6f4,
+//               M=128 N=128 K=64, operands in smem) and O_t += P_t [V^T;1]^T
+//               (M=128 N=80 K=128, P read from TMEM); the 16 extra rows of
+//               ones in the V stage give the row sum l = sum P in O's
+//               columns 64..79, so the softmax never adds up P itself;
+//   warps 0..7  softmax, warpgroup t for tile t, one TMEM lane (= query row)
+//               per thread: row max, P = 2^(z*c2 - m2) -> e4m3 written back
+//               into TMEM over S, and O rescaled when the running max rises.
+// The two tiles ping-pong: while one warpgroup turns S into P the tensor core
+// works on the other tile.
+//
+// TMEM (512 columns): S0 [0,128)  S1 [128,256)  O0 [256,336)  O1 [336,416).
+#include <math.h>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace sdm {
+namespace {
+
+constexpr int kStages = 4;
+constexpr int kTiles = 2;                 // query tiles per CTA
+constexpr int kSoftmaxWarps = 4 * kTiles;
+constexpr int kProducerWarp = kSoftmaxWarps;
+constexpr int kMmaWarp = kSoftmaxWarps + 1;
+constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+
+constexpr int kQBytes = kQTile * kHeadDim;        // 8 KB, 64-byte rows
+constexpr int kKBytes = kKvTile * kHeadDim;       // 8 KB, 64-byte rows
+constexpr int kVRows = kHeadDim + 16;             // V^T rows + 16 rows of ones
+constexpr int kVBytes = kVRows * kKvTile;         // 10 KB, 128-byte rows
+constexpr int kVLoadBytes = kHeadDim * kKvTile;   // 8 KB loaded by TMA
+
+constexpr uint32_t kTmemCols = 512;
+__device__ __forceinline__ uint32_t s_col(int t) { return 128u * t; }
+__device__ __forceinline__ uint32_t o_col(int t) { return 256u + 80u * t; }
+
+constexpr long long kWaitLimit = 1LL << 31;   // ~1 s of SM clock: no legitimate wait comes close
+constexpr long long kDrainLimit = 1LL << 24;  // teardown waits for copies in flight
+
+struct __align__(1024) Smem {
+  uint8_t q[kTiles][kQBytes];
+  uint8_t k[kStages][kKBytes];
+  uint8_t v[kStages][kVBytes];
+  uint64_t q_full;
+  uint64_t k_full[kStages];
+  uint64_t v_full[kStages];
+  uint64_t kv_empty[kStages];
+  uint64_t s_full[kTiles];
+  uint64_t p_full[kTiles];
+  uint64_t o_full[kTiles];
+  uint64_t drain;
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+};
+
+struct KParams {
+  int32_t BH, H;
+  int64_t T, N;
+  int64_t n_pairs, n_splits, split_keys;
+  const float* scales;  // [3][BH]
+  __half* out;
+  float* part_acc;
+  float* part_ml;
+  uint32_t* err;
+};
+
+__device__ __forceinline__ void raise_abort(Smem& s, uint32_t* err, uint32_t code) {
+  atomicOr(err, code);
+  *reinterpret_cast<volatile uint32_t*>(&s.abort_flag) = 1u;
+}
+
+// Bounded wait used during teardown: ignores the abort flag.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kDrainLimit) {
+      atomicOr(err, kErrTimeoutDrain);
+      return;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    icl_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const KParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const volatile uint32_t* abort_flag = &s.abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- which tile pair, which key range
+  const int64_t blk = blockIdx.x;
+  const int64_t pair = blk % p.n_pairs;
+  const int64_t rest = blk / p.n_pairs;
+  const int64_t split = rest % p.n_splits;
+  const int64_t bh = rest / p.n_splits;
+  const int64_t row0 = pair * (kTiles * kQTile);
+  const int64_t kv_begin = (p.n_splits > 1) ? split * p.split_keys : 0;
+  const int64_t kv_end = (p.n_splits > 1) ? min(p.N, kv_begin + p.split_keys) : p.N;
+  const int n_tiles = static_cast<int>((kv_end - kv_begin + kKvTile - 1) / kKvTile);
+
+  // ---- set-up
+  if (threadIdx.x == 0) {
+    mbar_init(&s.q_full, 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&s.k_full[i], 1);
+      mbar_init(&s.v_full[i], 1);
+      mbar_init(&s.kv_empty[i], 1);
+    }
+    for (int t = 0; t < kTiles; ++t) {
+      mbar_init(&s.s_full[t], 1);
+      mbar_init(&s.p_full[t], 4);  // one arrival per softmax warp
+      mbar_init(&s.o_full[t], 1);
+    }
+    mbar_init(&s.drain, 1);
+    s.abort_flag = 0u;
+    fence_mbar_init();
+  }
+  // rows 64..79 of every V stage hold e4m3 1.0 (0x38): the row-sum block
+  for (int i = threadIdx.x; i < kStages * (16 * kKvTile / 4); i += kThreads) {
+    const int st = i / (16 * kKvTile / 4), w = i % (16 * kKvTile / 4);
+    reinterpret_cast<uint32_t*>(s.v[st] + kVLoadBytes)[w] = 0x38383838u;
+  }
+  fence_proxy_async_smem();
+  if (warp == kMmaWarp) {
+    tmem_alloc(&s.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+
+  if (warp == kProducerWarp) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(&s.q_full, kTiles * kQBytes);
+      for (int t = 0; t < kTiles; ++t)
+        tma_load_3d(s.q[t], &tm_q, &s.q_full, 0, static_cast<int32_t>(row0 + t * kQTile), static_cast<int32_t>(bh));
+      int issued = 0;
+      for (int it = 0; it < n_tiles; ++it) {
+        const int st = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        if (!mbar_wait(&s.kv_empty[st], ph ^ 1u, abort_flag, kWaitLimit)) {
+          raise_abort(s, p.err, kErrTimeoutEmpty);
+          break;
+        }
+        const int32_t key0 = static_cast<int32_t>(kv_begin + (int64_t)it * kKvTile);
+        mbar_arrive_expect_tx(&s.k_full[st], kKBytes);
+        tma_load_3d(s.k[st], &tm_k, &s.k_full[st], 0, key0, static_cast<int32_t>(bh));
+        mbar_arrive_expect_tx(&s.v_full[st], kVLoadBytes);
+        tma_load_3d(s.v[st], &tm_v, &s.v_full[st], key0, 0, static_cast<int32_t>(bh));
+        issued = it + 1;
+      }
+      // teardown: every copy issued must have landed before the CTA exits
+      drain_wait(&s.q_full, 0, p.err);
+      for (int it = issued > kStages ? issued - kStages : 0; it < issued; ++it) {
+        drain_wait(&s.k_full[it % kStages], (it / kStages) & 1, p.err);
+        drain_wait(&s.v_full[it % kStages], (it / kStages) & 1, p.err);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_e4m3_f32(kQTile, kKvTile);
+      const uint32_t idesc_o = idesc_e4m3_f32(kQTile, kVRows);
+      auto issue_qk = [&](int t, int st) {
+        const uint32_t a0 = smem_u32(s.q[t]), b0 = smem_u32(s.k[st]);
+#pragma unroll
+        for (int ks = 0; ks < kHeadDim / 32; ++ks)
+          mma_e4m3_ss(tmem + s_col(t), smem_desc_kmajor(a0 + 32 * ks, 512, kSwizzle64B),
+                      smem_desc_kmajor(b0 + 32 * ks, 512, kSwizzle64B), idesc_s, ks > 0);
+      };
+      auto issue_pv = [&](int t, int st, bool acc) {
+        const uint32_t b0 = smem_u32(s.v[st]);
+#pragma unroll
+        for (int ks = 0; ks < kKvTile / 32; ++ks)
+          mma_e4m3_ts(tmem + o_col(t), tmem + s_col(t) + 8 * ks, smem_desc_kmajor(b0 + 32 * ks, 1024, kSwizzle128B),
+                      idesc_o, (acc || ks > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(&s.q_full, 0, abort_flag, kWaitLimit);
+      if (!ok) raise_abort(s, p.err, kErrTimeoutQ);
+      if (ok && n_tiles > 0) {
+        ok = mbar_wait(&s.k_full[0], 0, abort_flag, kWaitLimit);
+        if (!ok) raise_abort(s, p.err, kErrTimeoutKV);
+      }
+      if (ok && n_tiles > 0) {
+        tc_fence_after();
+        for (int t = 0; t < kTiles; ++t) {
+          issue_qk(t, 0);
+          mma_commit(&s.s_full[t]);
+        }
+      }
+      for (int it = 0; ok && it < n_tiles; ++it) {
+        const int st = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        const int nst = (it + 1) % kStages;
+        const uint32_t nph = ((it + 1) / kStages) & 1;
+        if (!mbar_wait(&s.v_full[st], ph, abort_flag, kWaitLimit)) {
+          raise_abort(s, p.err, kErrTimeoutKV);
+          ok = false;
+          break;
+        }
+        for (int t = 0; t < kTiles; ++t) {
+          if (!mbar_wait(&s.p_full[t], it & 1, abort_flag, kWaitLimit)) {
+            raise_abort(s, p.err, kErrTimeoutP);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_pv(t, st, it > 0);
+          if (t == kTiles - 1) mma_commit(&s.kv_empty[st]);
+          if (it + 1 < n_tiles) {
+            if (t == 0) {
+              if (!mbar_wait(&s.k_full[nst], nph, abort_flag, kWaitLimit)) {
+                raise_abort(s, p.err, kErrTimeoutKV);
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            issue_qk(t, nst);
+            mma_commit(&s.s_full[t]);
+          } else {
+            mma_commit(&s.o_full[t]);
+          }
+        }
+      }
+      // teardown: every MMA issued must complete before TMEM is released
+      mma_commit(&s.drain);
+      drain_wait(&s.drain, 0, p.err);
+    }
+  } else {
+    // ================================================================ softmax
+    const int t = warp >> 2;   // query tile
+    const int wq = warp & 3;   // TMEM lane quadrant
+    const uint32_t lane_base = static_cast<uint32_t>(32 * wq) << 16;
+    const uint32_t t_s = tmem + lane_base + s_col(t);
+    const uint32_t t_o = tmem + lane_base + o_col(t);
+    const float s_q = __ldg(p.scales + bh);
+    const float s_k = __ldg(p.scales + p.BH + bh);
+    const float s_v = __ldg(p.scales + 2 * p.BH + bh);
+    // c2 = s_q * s_k * log2(e) / sqrt(64): logits in base-2 units per raw z
+    const float c2 = __fmul_rn(__fmul_rn(s_q, s_k), 0.18033688011112042f);
+    float m_run = -INFINITY;  // running max of raw z
+    float m2 = -INFINITY;     // fp32(m_run * c2)
+    bool ok = true;
+    for (int it = 0; it < n_tiles; ++it) {
+      ok = mbar_wait(&s.s_full[t], it & 1, abort_flag, kWaitLimit);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (lane == 0) raise_abort(s, p.err, kErrTimeoutS);
+        break;
+      }
+      tc_fence_after();
+      uint32_t r[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(t_s + 32 * c, r[c]);
+      tmem_ld_wait();
+      const int64_t nvalid = kv_end - (kv_begin + (int64_t)it * kKvTile);
+      if (nvalid < kKvTile) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (32 * c + i >= nvalid) r[c][i] = __float_as_uint(-INFINITY);
+      }
+      float mt = m_run;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mt = fmaxf(mt, __uint_as_float(r[c][i]));
+      const bool up = mt > m_run;
+      const float m2_new = up ? __fmul_rn(mt, c2) : m2;
+      if (it > 0 && __any_sync(0xffffffffu, up)) {
+        // O and its row sum were accumulated against the old max: rescale.
+        const float alpha = up ? ex2_approx(__fsub_rn(m2, m2_new)) : 1.0f;
+        uint32_t o[32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          tmem_ld_32x32b_x32(t_o + 32 * c, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__fmul_rn(__uint_as_float(o[i]), alpha));
+          tmem_st_32x32b_x32(t_o + 32 * c, o);
+        }
+        uint32_t l;
+        tmem_ld_32x32b_x1(t_o + kHeadDim, l);
+        tmem_ld_wait();
+        tmem_st_32x32b_x1(t_o + kHeadDim, __float_as_uint(__fmul_rn(__uint_as_float(l), alpha)));
+      }
+      m_run = mt;
+      m2 = m2_new;
+      // P = 2^(fma(z, c2, -m2)) in (0, 1], four e4m3 codes per 32-bit column
+      uint32_t pw[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          const float p0 = ex2_approx(__fmaf_rn(__uint_as_float(r[c][4 * w + 0]), c2, -m2));
+          const float p1 = ex2_approx(__fmaf_rn(__uint_as_float(r[c][4 * w + 1]), c2, -m2));
+          const float p2 = ex2_approx(__fmaf_rn(__uint_as_float(r[c][4 * w + 2]), c2, -m2));
+          const float p3 = ex2_approx(__fmaf_rn(__uint_as_float(r[c][4 * w + 3]), c2, -m2));
+          pw[8 * c + w] = e4m3x2(p0, p1) | (e4m3x2(p2, p3) << 16);
+        }
+      tmem_st_32x32b_x32(t_s, pw);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.p_full[t]);
+    }
+    // ---- epilogue
+    if (ok && n_tiles > 0) {
+      ok = mbar_wait(&s.o_full[t], 0, abort_flag, kWaitLimit);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok && lane == 0) raise_abort(s, p.err, kErrTimeoutO);
+    }
+    if (ok && n_tiles > 0) {
+      tc_fence_after();
+      uint32_t o0[32], o1[32], l;
+      tmem_ld_32x32b_x32(t_o, o0);
+      tmem_ld_32x32b_x32(t_o + 32, o1);
+      tmem_ld_32x32b_x1(t_o + kHeadDim, l);
+      tmem_ld_wait();
+      const int64_t row = row0 + (int64_t)t * kQTile + 32 * wq + lane;
+      if (row < p.T) {
+        const float lf = __uint_as_float(l);
+        if (p.n_splits == 1) {
+          const int64_t b = bh / p.H, h = bh % p.H;
+          uint4* dst = reinterpret_cast<uint4*>(p.out + ((b * p.T + row) * p.H + h) * kHeadDim);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int e = 8 * v + 2 * k;
+              const float x0 = __uint_as_float(e < 32 ? o0[e] : o1[e - 32]);
+              const float x1 = __uint_as_float(e + 1 < 32 ? o0[e + 1] : o1[e + 1 - 32]);
+              const __half2 hv = __halves2half2(__float2half_rn(__fdiv_rn(__fmul_rn(x0, s_v), lf)),
+                                                __float2half_rn(__fdiv_rn(__fmul_rn(x1, s_v), lf)));
+              w[k] = *reinterpret_cast<const uint32_t*>(&hv);
+            }
+            dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        } else {
+          const int64_t prow = (split * p.BH + bh) * p.T + row;
+          float4* dst = reinterpret_cast<float4*>(p.part_acc + prow * kHeadDim);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            dst[v] = make_float4(__uint_as_float(o0[4 * v]), __uint_as_float(o0[4 * v + 1]),
+                                 __uint_as_float(o0[4 * v + 2]), __uint_as_float(o0[4 * v + 3]));
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            dst[8 + v] = make_float4(__uint_as_float(o1[4 * v]), __uint_as_float(o1[4 * v + 1]),
+                                     __uint_as_float(o1[4 * v + 2]), __uint_as_float(o1[4 * v + 3]));
+          reinterpret_cast<float2*>(p.part_ml)[prow] = make_float2(m2, lf);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------ split-KV reduce
+// One warp per (b, h, row): M2 = max_s m2_s; w_s = 2^(m2_s - M2);
+// O = (sum_s w_s acc_s) * s_v / (sum_s w_s l_s), splits in ascending order.
+__global__ void __launch_bounds__(256) splitkv_reduce_kernel(const float* __restrict__ part_acc,
+                                                             const float* __restrict__ part_ml, int64_t n_splits,
+                                                             int32_t BH, int32_t H, int64_t T,
+                                                             const float* __restrict__ scales, __half* __restrict__ out) {
+  const int64_t gw = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (gw >= (int64_t)BH * T) return;
+  const int64_t bh = gw / T, row = gw % T;
+  const float2* ml = reinterpret_cast<const float2*>(part_ml);
+  float M2 = -INFINITY;
+  for (int64_t sidx = 0; sidx < n_splits; ++sidx) M2 = fmaxf(M2, ml[(sidx * BH + bh) * T + row].x);
+  float L = 0.0f, a0 = 0.0f, a1 = 0.0f;
+  for (int64_t sidx = 0; sidx < n_splits; ++sidx) {
+    const int64_t prow = (sidx * BH + bh) * T + row;
+    const float2 e = ml[prow];
+    const float w = ex2_approx(__fsub_rn(e.x, M2));
+    const float2 acc = reinterpret_cast<const float2*>(part_acc + prow * kHeadDim)[lane];
+    L = __fmaf_rn(w, e.y, L);
+    a0 = __fmaf_rn(w, acc.x, a0);
+    a1 = __fmaf_rn(w, acc.y, a1);
+  }
+  const float s_v = __ldg(scales + 2 * BH + bh);
+  const int64_t b = bh / H, h = bh % H;
+  const __half2 hv = __halves2half2(__float2half_rn(__fdiv_rn(__fmul_rn(a0, s_v), L)),
+                                    __float2half_rn(__fdiv_rn(__fmul_rn(a1, s_v), L)));
+  reinterpret_cast<__half2*>(out + ((b * T + row) * H + h) * kHeadDim)[lane] = hv;
+}
+
+// ------------------------------------------------------------ host helpers
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 3-D uint8 tensor map: dims {d0, d1, d2} (d0 innermost), row stride s1 bytes,
+// plane stride s2 bytes, box {b0, b1, 1}.
+bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1, uint64_t s2,
+              uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {s1, s2};
+  const cuuint32_t box[3] = {b0, b1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8t, const AttnArgs& a,
+                             cudaStream_t st) {
+  const int64_t BH = (int64_t)a.B * a.H;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q8, kHeadDim, a.T, BH, kHeadDim, a.T * kHeadDim, kHeadDim, kQTile,
+                CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map(&tk, k8, kHeadDim, a.N, BH, kHeadDim, a.N * kHeadDim, kHeadDim, kKvTile,
+                CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map(&tv, v8t, a.ld_v, kHeadDim, BH, a.ld_v, a.ld_v * kHeadDim, kKvTile, kHeadDim,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  KParams p;
+  p.BH = static_cast<int32_t>(BH);
+  p.H = a.H;
+  p.T = a.T;
+  p.N = a.N;
+  p.n_pairs = (a.T + kTiles * kQTile - 1) / (kTiles * kQTile);
+  p.n_splits = a.n_splits;
+  p.split_keys = a.split_keys;
+  p.scales = a.scales;
+  p.out = a.out;
+  p.part_acc = a.part_acc;
+  p.part_ml = a.part_ml;
+  p.err = a.err;
+  const size_t smem = sizeof(Smem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(icl_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int64_t grid = p.n_pairs * p.n_splits * BH;
+  if (grid == 0) return cudaSuccess;
+  icl_attention_kernel<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_splitkv_reduce(const AttnArgs& a, cudaStream_t st) {
+  const int64_t BH = (int64_t)a.B * a.H;
+  const int64_t warps = BH * a.T;
+  if (warps == 0) return cudaSuccess;
+  const int64_t blocks = (warps * 32 + 255) / 256;
+  splitkv_reduce_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(a.part_acc, a.part_ml, a.n_splits,
+                                                                       static_cast<int32_t>(BH), a.H, a.T, a.scales,
+                                                                       a.out);
+  return cudaGetLastError();
+}
+
+}  // namespace sdm

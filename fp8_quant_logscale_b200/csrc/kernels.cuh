@@ -1,0 +1,80 @@
+// kernels.cuh -- launch wrappers shared by the C-ABI layer (api.cu) and the
+// kernel files.  Internal to the library; the public interface is sdm_fp8.h.
+#pragma once
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace sdm {
+
+constexpr int kHeadDim = 64;   // the only head dimension the kernels are built for
+constexpr int kKvTile = 128;   // keys per online-softmax block (one tcgen05 N=128 tile)
+constexpr int kQTile = 128;    // query rows per tensor-core tile (M=128)
+constexpr int64_t kSplitKeys = 16384;  // cached prediction: keys per split-KV chunk
+
+// Query-scaling parameters shared by the elementwise kernels.
+struct QScale {
+  bool enabled;        // false: the input already is q' (or is K / V)
+  float lam;           // fp32 ln(max(n,1)), evaluated on the host from the integer length
+  const float* c_h;    // [H] per-head coefficients (device)
+  const __half* gate;  // [B][rows][H] or nullptr (LogScale)
+};
+
+// Tensor-wide problem description for the elementwise kernels.
+struct RowsDesc {
+  const __half* x;     // [B][rows][H][64]
+  int32_t B, H;
+  int64_t rows;        // rows per batch in x's layout
+};
+
+cudaError_t launch_qscale(const __half* q, __half* out, int32_t B, int64_t rows, int32_t H, QScale qs,
+                          cudaStream_t st);
+
+// amax words: [3][B][H] uint32 (float bits, values >= 0).  Must be zeroed first.
+cudaError_t launch_context_amax(RowsDesc q, QScale qs, RowsDesc k, RowsDesc v, int64_t n_ctx, uint32_t* amax,
+                                cudaStream_t st);
+
+// scales[3][B][H] = amax/448 (1 where amax == 0); from the amax words.
+cudaError_t launch_scales_from_amax(const uint32_t* amax, int32_t BH, float* scales, cudaStream_t st);
+
+// Row-major quantisation: dst[b][h][r][64] = e4m3(qscale?(x[b][r][h][:]) / scale[b*H+h]),
+// rows [0, n_rows) of x; dst has dst_rows rows per (b, h).
+cudaError_t launch_quantize_rows(RowsDesc x, QScale qs, int64_t n_rows, const float* scale, uint8_t* dst,
+                                 int64_t dst_rows, cudaStream_t st);
+
+// Transposed quantisation for V: dst[b][h][e][ld] for keys [0, n_ctx), zeros in [n_ctx, ld).
+cudaError_t launch_quantize_vt(RowsDesc v, int64_t n_ctx, const float* scale, uint8_t* dst, int64_t ld,
+                               cudaStream_t st);
+
+// ---------------------------------------------------------------- attention
+struct AttnArgs {
+  int32_t B, H;
+  int64_t T;           // query rows per (b, h) in the Q8 layout
+  int64_t N;           // context keys
+  int64_t ld_v;        // V8 transposed row length (keys), multiple of 128
+  const float* scales; // [3][B][H]: s_q, s_k, s_v
+  int64_t n_splits;    // 1: single pass, final output; >1: split-KV partials
+  int64_t split_keys;  // keys per split (multiple of kKvTile) when n_splits > 1
+  __half* out;         // final: [B][T][H][64] fp16
+  float* part_acc;     // split: [S][B*H][T][64]
+  float* part_ml;      // split: [S][B*H][T][2] (m2, l)
+  uint32_t* err;       // device error word
+};
+
+// Builds the tensor maps and launches the tcgen05 attention kernel.
+cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8t, const AttnArgs& a,
+                             cudaStream_t st);
+// Combines split-KV partials in split order into the fp16 output.
+cudaError_t launch_splitkv_reduce(const AttnArgs& a, cudaStream_t st);
+
+// Device error word bits.
+constexpr uint32_t kErrTimeoutQ = 1u << 0;
+constexpr uint32_t kErrTimeoutKV = 1u << 1;
+constexpr uint32_t kErrTimeoutS = 1u << 2;
+constexpr uint32_t kErrTimeoutP = 1u << 3;
+constexpr uint32_t kErrTimeoutO = 1u << 4;
+constexpr uint32_t kErrTimeoutEmpty = 1u << 5;
+constexpr uint32_t kErrTimeoutDrain = 1u << 6;
+
+}  // namespace sdm

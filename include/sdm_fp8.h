@@ -1,0 +1,217 @@
+/*
+ * sdm_fp8.h -- C ABI of the B200 (sm_100a) FP8 in-context-learning attention
+ * layer: fused LogScale/GatedLogScale query scaling, FP8 e4m3 quantisation
+ * with context-derived per-head scales, FP8 flash attention, and cached
+ * prediction against a resident FP8 K/V cache with split-KV.
+ *
+ * Sources (web pages, cited by title and section):
+ *   "Fuse shared-length query scaling during inference" (structured-data-models
+ *     PR #1168), "Problem identified" and "Solution": LogScale/GatedLogScale,
+ *     float32 length arithmetic, per-head conversion, query multiply and gate
+ *     fused, every eager rounding boundary preserved.
+ *   "[FP8 3/4] Integrate FP8 attention and caching into TabICLv2"
+ *     (structured-data-models PR #879), opening section and usage example:
+ *     FP8 attention of the intermediate ICL layers, Q scales derived from the
+ *     context only, fit once / predict many with a quantised K/V cache, and a
+ *     RuntimeError when a cache is misused (here: SDM_ERR_CACHE_MISMATCH).
+ *   "[TRTLLM-15160][feat] ... make trtllm::kda_decode inplace-only"
+ *     (TensorRT-LLM PR #18375), walkthrough: results go only into
+ *     caller-owned output storage, checked for device, dtype and layout before
+ *     launch.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are device memory of the CURRENT CUDA device,
+ *     allocated and owned by the caller, 16-byte aligned (workspace: 256-byte
+ *     aligned), row-major and contiguous in the layout stated.  The library
+ *     allocates nothing and writes only to the outputs, the cache buffers and
+ *     the workspace it is given.
+ *   - fp16 data is IEEE binary16; e4m3 data is OCP FP8 E4M3 ("fn": max 448,
+ *     0x7F/0xFF NaN) stored one code per byte.
+ *   - head_dim must be 64 (SDM_ERR_UNSUPPORTED otherwise); 1 <= heads <= 128.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and the call returns without synchronising.  Argument errors are
+ *     reported before anything is enqueued.  A bounded in-kernel wait that
+ *     gives up ORs a flag into the error word (the first 4 bytes of the
+ *     workspace); sdm_sync_status() reports it as SDM_ERR_TIMEOUT and clears
+ *     it.  A workspace's first 256 bytes must be zero before its first use.
+ *   - Layout symbols: B batch, N context rows, M query rows, T = N + M,
+ *     H heads, d = 64.  Context rows are rows [0, N) of every row-indexed
+ *     tensor; query rows are [N, T).
+ */
+#ifndef SDM_FP8_H
+#define SDM_FP8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SDM_OK = 0,
+  SDM_ERR_INVALID_ARG = 1,     /* null pointer, bad size, misaligned pointer */
+  SDM_ERR_UNSUPPORTED = 2,     /* head_dim != 64, heads outside [1,128], sizes past the kernels' limits */
+  SDM_ERR_WORKSPACE = 3,       /* workspace missing or smaller than sdm_workspace_size() */
+  SDM_ERR_DEVICE_MISMATCH = 4, /* a pointer is not device memory of the current device */
+  SDM_ERR_CACHE_MISMATCH = 5,  /* cache shape/device disagrees with the call, or cache not filled */
+  SDM_ERR_TIMEOUT = 6,         /* an in-kernel bounded wait gave up (from sdm_sync_status) */
+  SDM_ERR_CUDA = 7             /* a CUDA runtime call or launch failed */
+} sdm_status;
+
+/* Operations, for sdm_workspace_size(). */
+typedef enum {
+  SDM_OP_QUANTIZE_CONTEXT = 0,
+  SDM_OP_ICL_ATTENTION = 1,
+  SDM_OP_CACHED_ATTENTION = 2
+} sdm_op;
+
+/* Keys per online-softmax block and per cached-prediction split-KV chunk.
+ * The chunk boundaries of the cached path depend on the context length only,
+ * so a query's cached prediction does not depend on how queries are batched. */
+#define SDM_KV_TILE 128
+#define SDM_SPLIT_KEYS 16384
+
+/*
+ * FP8 K/V cache: the fitted state that cached prediction reads (the analogue
+ * of the pages' quantised KV cache entry).  The caller allocates the three
+ * buffers with the sizes from sdm_cache_layout() on one device and fills in
+ * every field; sdm_fp8_quantize_context() or sdm_icl_attention() writes the
+ * contents and sets `filled` to 1.
+ *   k8     [B][H][N][64]   e4m3, keys row-major
+ *   v8t    [B][H][64][ld_v] e4m3, V transposed (keys contiguous);
+ *          ld_v = N rounded up to a multiple of 128; keys [N, ld_v) are zero
+ *   scales [3][B][H]        fp32: s_q, s_k, s_v (amax/448 over context rows)
+ */
+typedef struct {
+  uint8_t* k8;
+  uint8_t* v8t;
+  float* scales;
+  int64_t n_ctx;
+  int64_t ld_v;
+  int32_t batch;
+  int32_t heads;
+  int32_t head_dim;
+  int32_t device;
+  int32_t filled;
+} sdm_fp8_cache;
+
+/* Human-readable name of a status code (static storage). */
+const char* sdm_status_string(sdm_status status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int32_t sdm_version(void);
+
+/*
+ * Byte sizes of the three cache buffers for B x N x H x d, and ld_v.
+ * Returns SDM_ERR_INVALID_ARG / SDM_ERR_UNSUPPORTED for bad shapes.
+ */
+sdm_status sdm_cache_layout(int32_t batch, int64_t n_ctx, int32_t heads, int32_t head_dim, size_t* k8_bytes,
+                            size_t* v8t_bytes, size_t* scales_bytes, int64_t* ld_v);
+
+/*
+ * Workspace bytes `op` needs for these sizes (0 on invalid sizes).  For
+ * SDM_OP_ICL_ATTENTION, keep_cache == 0 means the call gets no cache and the
+ * workspace also holds K8/V8/scales; for the other ops keep_cache is ignored.
+ * n_query is M for SDM_OP_CACHED_ATTENTION.
+ */
+size_t sdm_workspace_size(sdm_op op, int32_t batch, int64_t n_ctx, int64_t n_query, int32_t heads,
+                          int32_t head_dim, int32_t keep_cache);
+
+/*
+ * Step 1 -- fused LogScale / GatedLogScale ("Fuse shared-length query scaling
+ * during inference", "Solution").  For every row r, head h and element e:
+ *   lam = fp32 ln(max(n_len, 1))            (the shared integer key length)
+ *   s_h = fp16(fp32(c_h[h] * lam))           (per-head conversion)
+ *   q1  = fp16(fp32(q * s_h))
+ *   gated: u = fp16(tanh(gate)), w = fp16(1 + u), q_out = fp16(q1 * w)
+ * with one round-to-nearest-even per eager operation.
+ *   q, q_out  [B][rows][H][d] fp16 (may alias exactly: in place)
+ *   c_h       [H] fp32, device
+ *   gate      [B][rows][H] fp16, or NULL for LogScale
+ *   n_len     >= 1
+ */
+sdm_status sdm_qscale_fused(const void* q, void* q_out, int32_t batch, int64_t rows, int32_t heads,
+                            int32_t head_dim, int64_t n_len, const float* c_h, const void* gate, void* stream);
+
+/*
+ * Step 2 -- context-derived FP8 quantisation ("[FP8 3/4] ...", opening
+ * section).  Per (b, h): s_X = amax(|X| over context rows [0, N) and all d)
+ * / 448 for X in {Q', K, V} (1 if the amax is 0), then
+ * X8 = e4m3_rne_satfinite(fp32(X) / s_X) with IEEE division.
+ *   q_scaled  [B][T][H][d] fp16, already query-scaled (step 1); T = N + M
+ *   k, v      [B][N][H][d] fp16 (context rows only)
+ *   q8        [B][H][T][d] e4m3 out; query rows use the context scale and saturate
+ *   cache     out: k8, v8t, scales written, `filled` set; shape fields must match
+ *   ws        >= sdm_workspace_size(SDM_OP_QUANTIZE_CONTEXT, ...) bytes
+ */
+sdm_status sdm_fp8_quantize_context(const void* q_scaled, const void* k, const void* v, int32_t batch,
+                                    int64_t n_ctx, int64_t n_query, int32_t heads, int32_t head_dim, uint8_t* q8,
+                                    sdm_fp8_cache* cache, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Step 3 alone -- FP8 flash attention of already-quantised rows to the cache
+ * ("[FP8 3/4] ...", opening section).  For each row i and head h, over keys
+ * j < N of the cache, in 128-key blocks:
+ *   z_j = sum_e q8[e]*k8_j[e] (fp32 tensor-core accumulation)
+ *   c2 = fp32(fp32(s_q*s_k) * fp32(log2(e)/8));  m = running max z;
+ *   P_j = e4m3(2^(fma(z_j, c2, -fp32(m*c2))))  -- probabilities in (0, 1]
+ *   l = sum_j P_j, acc = sum_j P_j * v8_j (rescaled by 2^(m2_old - m2_new)
+ *   whenever the running max rises); out = fp16(acc * s_v / l).
+ *   q8     [B][H][rows][d] e4m3
+ *   cache  filled FP8 cache (k8, v8t, scales)
+ *   out    [B][rows][H][d] fp16
+ *   split  0: one pass over all keys; 1: split-KV in SDM_SPLIT_KEYS chunks
+ *          combined in chunk order (the cached-prediction arithmetic)
+ *   ws     >= sdm_workspace_size(SDM_OP_CACHED_ATTENTION, B, N, rows, ...)
+ */
+sdm_status sdm_fp8_attention(const uint8_t* q8, int32_t batch, int64_t rows, const sdm_fp8_cache* cache, void* out,
+                             int32_t split, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Steps 1-3 -- one call of the FP8 ICL attention layer ("model(context,
+ * labels, queries)" on "[FP8 3/4] ...").  Query scaling with n = N is fused
+ * into the amax and quantisation passes; context rows attend to all context
+ * rows (themselves included) and query rows attend to the context rows.
+ *   q     [B][T][H][d] fp16 (raw, before query scaling), T = N + M
+ *   k, v  [B][N][H][d] fp16
+ *   c_h   [H] fp32 device;  gate [B][T][H] fp16 or NULL (LogScale)
+ *   out   [B][T][H][d] fp16
+ *   cache NULL: the FP8 K/V and scales live in the workspace and are
+ *         discarded; non-NULL: "fit" -- they are written to the cache's
+ *         buffers, which the caller then reuses for sdm_cached_attention.
+ *   ws    >= sdm_workspace_size(SDM_OP_ICL_ATTENTION, ..., cache != NULL)
+ */
+sdm_status sdm_icl_attention(const void* q, const void* k, const void* v, int32_t batch, int64_t n_ctx,
+                             int64_t n_query, int32_t heads, int32_t head_dim, const float* c_h, const void* gate,
+                             void* out, sdm_fp8_cache* cache, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Step 4 -- cached prediction ("model.predict(queries)" after "model.fit" on
+ * "[FP8 3/4] ...").  The M query rows are query-scaled with n = cache->n_ctx,
+ * quantised with the cache's context-derived s_q, and attend to the cache's
+ * keys with split-KV (SDM_SPLIT_KEYS-key chunks, a fixed-order combine), so a
+ * query's output is identical however the queries are batched.
+ *   q    [B][M][H][d] fp16 raw;  gate [B][M][H] fp16 or NULL;  c_h [H] fp32
+ *   out  [B][M][H][d] fp16
+ *   ws   >= sdm_workspace_size(SDM_OP_CACHED_ATTENTION, B, cache->n_ctx, M, ...)
+ * Returns SDM_ERR_CACHE_MISMATCH if the cache is unfilled, on another device,
+ * or its batch/heads/head_dim differ from the call's.
+ */
+sdm_status sdm_cached_attention(const void* q, int32_t batch, int64_t n_query, int32_t heads, int32_t head_dim,
+                                const sdm_fp8_cache* cache, const float* c_h, const void* gate, void* out, void* ws,
+                                size_t ws_bytes, void* stream);
+
+/*
+ * Wait for `stream`, then read and clear the device error word at the head of
+ * a workspace used by the calls above.  Returns SDM_OK, SDM_ERR_TIMEOUT (an
+ * in-kernel wait gave up; `*flags` gets the raw bits if flags != NULL) or
+ * SDM_ERR_CUDA (an asynchronous CUDA error surfaced).
+ */
+sdm_status sdm_sync_status(void* ws, void* stream, uint32_t* flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDM_FP8_H */

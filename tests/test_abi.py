@@ -1,0 +1,78 @@
+"""The C-ABI library builds, loads and exports every symbol include/sdm_fp8.h
+declares; argument errors come back as status codes before any CUDA work
+(no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from fp8_quant_logscale_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sdm_fp8.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return binding.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sdm_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_four_layer_calls():
+    syms = declared_symbols()
+    for name in ("sdm_qscale_fused", "sdm_fp8_quantize_context", "sdm_icl_attention", "sdm_cached_attention"):
+        assert name in syms
+
+
+def test_every_declared_symbol_is_exported(L):
+    syms = declared_symbols()
+    assert set(syms) == set(binding.EXPORTS)
+    for name in syms:
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code, name in binding.STATUS_NAMES.items():
+        assert L.sdm_status_string(code).decode().startswith(name)
+    assert L.sdm_version() == 100
+
+
+def test_cache_layout_and_workspace_sizes(L):
+    kb, vb, sb, ld = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_int64()
+    st = L.sdm_cache_layout(2, 1000, 3, 64, ctypes.byref(kb), ctypes.byref(vb), ctypes.byref(sb), ctypes.byref(ld))
+    assert st == 0 and ld.value == 1024
+    assert kb.value == 2 * 3 * 1000 * 64 and vb.value == 2 * 3 * 64 * 1024 and sb.value == 3 * 2 * 3 * 4
+    assert L.sdm_cache_layout(1, 1000, 3, 32, None, None, None, None) == 2       # d != 64
+    assert L.sdm_cache_layout(1, 0, 3, 64, None, None, None, None) == 1          # N < 1
+    assert L.sdm_cache_layout(1, 10, 129, 64, None, None, None, None) == 2       # too many heads
+    w_icl = binding.workspace_size(binding.OP_ICL_ATTENTION, 1, 16384, 1024, 8, keep_cache=True)
+    w_icl_nc = binding.workspace_size(binding.OP_ICL_ATTENTION, 1, 16384, 1024, 8, keep_cache=False)
+    assert w_icl >= 8 * 17408 * 64 and w_icl_nc >= w_icl + 2 * 8 * 16384 * 64
+    w_c = binding.workspace_size(binding.OP_CACHED_ATTENTION, 1, 524288, 1024, 8)
+    assert w_c >= 32 * 8 * 1024 * 66 * 4                                           # 32 split-KV partials
+    assert L.sdm_workspace_size(0, 1, 100, 0, 8, 32, 1) == 0
+    assert L.sdm_workspace_size(7, 1, 100, 0, 8, 64, 1) == 0
+
+
+def test_shape_errors_before_any_cuda_call(L):
+    assert L.sdm_qscale_fused(None, None, 1, 10, 4, 32, 10, None, None, None) == 2
+    assert L.sdm_qscale_fused(None, None, 0, 10, 4, 64, 10, None, None, None) == 1
+    assert L.sdm_icl_attention(None, None, None, 1, 0, 5, 4, 64, None, None, None, None, None, 0, None) == 1
+    assert L.sdm_icl_attention(None, None, None, 1, 10, 5, 4, 48, None, None, None, None, None, 0, None) == 2
+    assert L.sdm_cached_attention(None, 1, 5, 4, 64, None, None, None, None, None, 0, None) == 1
+    assert L.sdm_fp8_attention(None, 1, 5, None, None, 0, None, 0, None) == 1
+    assert L.sdm_sync_status(None, None, None) == 1
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_no_device_reports_cuda_error(L):
+    # valid shapes, no GPU: the device query fails and nothing is launched
+    assert L.sdm_qscale_fused(None, None, 1, 10, 4, 64, 10, None, None, None) == 7

@@ -1,0 +1,108 @@
+"""GPU parity of steps 1-3 (one call of the FP8 ICL attention layer) against the oracle.
+
+FP8 tensors and scales are compared bit for bit; attention outputs within the
+specification's gates (max |d| 2e-2, mean |d| 1e-3), where the oracle adds an
+allowance only for keys whose probability sits within relative 1e-4 of an
+e4m3 rounding midpoint (either code is a correct result there).  The error
+against exact attention is printed for the record.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from fp8_quant_logscale_b200.workloads import WORKLOADS, make_inputs
+from parity import DELTA, dev, gate, host
+
+pytestmark = pytest.mark.gpu
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+LOG2E = 1.4426950408889634
+
+
+def test_golden_worked_example_on_gpu(cuda_lib):
+    """Three keys whose probabilities are 1/4, 1/2, 1: the output is exactly 3."""
+    k2 = np.float32(LOG2E / 8.0)
+    sk = np.float32(1.0) / k2
+    for cand in (sk, np.nextafter(sk, np.float32(0)), np.nextafter(sk, np.float32(1e9))):
+        if np.float32(cand * k2) == np.float32(1.0):
+            sk = cand
+            break
+    cache = cuda_lib.FP8Cache(1, 3, 1, "cuda")
+    k8 = np.stack([np.full(64, c, np.uint8) for c in (0x00, 0x08, 0x10)])[None, None]
+    v8t = np.zeros((1, 1, 64, cache.ld_v), np.uint8)
+    v8t[..., :3] = np.array([0x38, 0x40, 0x48], np.uint8)
+    cache.k8.copy_(dev(k8))
+    cache.v8t.copy_(dev(v8t))
+    cache.scales.copy_(dev(np.array([1.0, sk, 1.0], np.float32).reshape(3, 1, 1)))
+    cache.struct.filled = 1
+    q8 = dev(np.full((1, 1, 5, 64), 0x38, np.uint8))
+    for split in (False, True):
+        out = host(cuda_lib.fp8_attention(q8, cache, split=split)).astype(np.float64)
+        assert (out == 3.0).all(), (split, out[0, 0, 0, :4])
+
+
+def _layer_case(cuda_lib, orc, inp, gated=False, rows=None, report=""):
+    B, N, M, H = inp["B"], inp["N"], inp["M"], inp["H"]
+    g = inp["gate"] if gated else None
+    cache = cuda_lib.FP8Cache(B, N, H, "cuda")
+    ws = cuda_lib.new_workspace(cuda_lib.workspace_size(1, B, N, M, H, keep_cache=True), "cuda")
+    out = cuda_lib.icl_attention(dev(inp["q"]), dev(inp["k"]), dev(inp["v"]), N, dev(inp["c_h"]), dev(g),
+                                 cache=cache, ws=ws)
+    st, flags = cuda_lib.sync_status(ws)
+    assert st == 0 and flags == 0, (st, flags)
+    # FP8 intermediates: bit-exact
+    qs = orc.qscale(inp["q"], N, inp["c_h"], g)
+    s_q, s_k, s_v = (orc.context_scales(x, N) for x in (qs, inp["k"], inp["v"]))
+    sc = host(cache.scales)
+    assert (sc[0] == s_q).all() and (sc[1] == s_k).all() and (sc[2] == s_v).all()
+    k8, v8 = orc.quantize(inp["k"], s_k), orc.quantize(inp["v"], s_v)
+    assert (host(cache.k8) == k8).all()
+    assert (host(cache.v8t)[..., :N] == v8.transpose(0, 1, 3, 2)).all()
+    q8 = orc.quantize(qs, s_q)
+    o16, o, allow = orc.attention(q8, k8, v8, s_q, s_k, s_v, rows=rows, delta=DELTA)
+    got = host(out) if rows is None else host(out)[:, rows]
+    stats = gate(got, o, allow, report)
+    exact = orc.attention_exact(qs, inp["k"], inp["v"], rows=rows)
+    e = got.astype(np.float64) - exact
+    stats["vs_exact_rel_rms"] = float(np.sqrt((e ** 2).mean() / (exact ** 2).mean()))
+    print(f"\n{report}: {stats}")
+    return stats
+
+
+@pytest.mark.parametrize("B,N,M,H", [(1, 1024, 128, 4), (2, 1000, 77, 3), (1, 1, 5, 2), (1, 300, 0, 1),
+                                     (1, 129, 300, 5)])
+def test_layer_small_full_parity(cuda_lib, orc, B, N, M, H):
+    inp = make_inputs(WORKLOADS["icl_n1k_m128_h4"], n_ctx=N, n_query=M, heads=H, batch=B)
+    _layer_case(cuda_lib, orc, inp, report=f"B{B} N{N} M{M} H{H}")
+
+
+def test_layer_gated_outliers_small(cuda_lib, orc):
+    inp = make_inputs(WORKLOADS["icl_n128k_m1k_h8_gated"], n_ctx=2048, n_query=200)
+    _layer_case(cuda_lib, orc, inp, gated=True, report="gated N2048")
+
+
+def _sample_rows(N, M, n_ctx_rows, n_q_rows, seed):
+    rng = np.random.default_rng(seed)
+    ctx = rng.choice(N, min(N, n_ctx_rows), replace=False)
+    qry = N + rng.choice(M, min(M, n_q_rows), replace=False)
+    return np.sort(np.concatenate([ctx, qry])).astype(np.int64)
+
+
+def test_layer_16k_sampled(cuda_lib, orc):
+    w = WORKLOADS["icl_n16k_m1k_h8"]
+    inp = make_inputs(w)
+    _layer_case(cuda_lib, orc, inp, rows=_sample_rows(w.n_ctx, w.n_query, 256, 256, 2), report="16K")
+
+
+def test_layer_128k_gated_sampled(cuda_lib, orc):
+    w = WORKLOADS["icl_n128k_m1k_h8_gated"]
+    inp = make_inputs(w)
+    _layer_case(cuda_lib, orc, inp, gated=True, rows=_sample_rows(w.n_ctx, w.n_query, 128, 128, 3),
+                report="128K gated")
+
+
+def test_layer_512k_sampled(cuda_lib, orc):
+    w = WORKLOADS["icl_n512k_m1k_h8"]
+    inp = make_inputs(w)
+    _layer_case(cuda_lib, orc, inp, rows=_sample_rows(w.n_ctx, w.n_query, 64, 128, 4), report="512K")

@@ -1,0 +1,39 @@
+"""GPU parity of step 2 (context-derived scales and e4m3 quantisation): scales,
+Q8, K8 and V8 (transposed layout, zero padding) bit-exact against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+from fp8_quant_logscale_b200.workloads import WORKLOADS, make_inputs
+from parity import dev, host
+
+pytestmark = pytest.mark.gpu
+
+
+def _check(cuda_lib, orc, q_scaled, k, v, N):
+    B, T, H, _ = q_scaled.shape
+    q8, cache = cuda_lib.fp8_quantize_context(dev(q_scaled), dev(k), dev(v), N)
+    torch.cuda.synchronize()
+    assert cache.filled
+    s_q, s_k, s_v = (orc.context_scales(x, N) for x in (q_scaled, k, v))
+    sc = host(cache.scales)
+    assert (sc[0] == s_q).all() and (sc[1] == s_k).all() and (sc[2] == s_v).all()
+    assert (host(q8) == orc.quantize(q_scaled, s_q)).all()
+    assert (host(cache.k8) == orc.quantize(k, s_k)).all()
+    v8t = host(cache.v8t)
+    want_v = orc.quantize(v, s_v)                        # [B,H,N,d]
+    assert (v8t[..., :N] == want_v.transpose(0, 1, 3, 2)).all()
+    assert (v8t[..., N:] == 0).all()
+
+
+@pytest.mark.parametrize("B,N,M,H", [(1, 1024, 128, 4), (2, 1000, 77, 3), (1, 1, 0, 2), (1, 130, 1, 8)])
+def test_quantize_bit_exact(cuda_lib, orc, B, N, M, H):
+    inp = make_inputs(WORKLOADS["icl_n16k_m1k_h8"], n_ctx=N, n_query=M, heads=H, batch=B)
+    qs = orc.qscale(inp["q"], N, inp["c_h"])
+    _check(cuda_lib, orc, qs, inp["k"], inp["v"], N)
+
+
+def test_quantize_with_outliers(cuda_lib, orc):
+    inp = make_inputs(WORKLOADS["icl_n128k_m1k_h8_gated"], n_ctx=8192, n_query=256)
+    qs = orc.qscale(inp["q"], 8192, inp["c_h"], inp["gate"])
+    _check(cuda_lib, orc, qs, inp["k"], inp["v"], 8192)
