@@ -1,0 +1,369 @@
+"""Benchmark of the FP8 in-context-learning attention layer on B200.
+
+One step = one pass of the whole hot path on the 512K-context workload:
+  fit:     sdm_icl_attention -- LogScale query scaling fused into the context
+           amax and e4m3 quantisation passes, then FP8 self + cross attention
+           of all 525,312 rows over 524,288 context keys, keeping the FP8 cache;
+  predict: sdm_cached_attention -- 1,024 new queries against that resident
+           524,288-row FP8 K/V cache with split-KV.
+Metric: FP8 attention TFLOP/s (algorithmic 4*d*H*rows*N per attention, both
+attentions of the step, divided by the step's device time), with the cached
+prediction's microseconds and the fraction of the FP8 tensor peak alongside.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU (torchrun): every rank runs its own independent problem (another
+estimator: different seed), no collective on the data path; value = all
+ranks' FLOPs / the slowest rank's time ("scaling": "weak").
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "FP8 ICL attention TFLOP/s at 128K/512K ctx (% FP8 peak); cached-predict us"
+DEFAULT_WORKLOAD = "icl_n512k_m1k_h8"
+CACHED_WORKLOAD = "cached_n512k_m1k_h8"
+FP8_NOMINAL_TFLOPS = 4500.0
+BF16_NOMINAL_TFLOPS = 2250.0
+
+
+def attn_flops(rows: int, n_ctx: int, heads: int, d: int = 64) -> float:
+    """Algorithmic FLOPs of one attention: S = QK^T and O = PV, 2*d each per (row, key, head)."""
+    return 4.0 * d * heads * rows * n_ctx
+
+
+# ------------------------------------------------------------------ ranks
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def init_dist(backend: str):
+    import datetime
+
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+    return rank, world
+
+
+def reduce_max(value: float, device) -> float:
+    """Max of a float over all ranks (the identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.barrier()
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"sdm_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        try:
+            rows = [ln.split(",") for ln in open(self.path) if ln.strip()]
+        except OSError:
+            rows = []
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows]
+        reasons = set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            for name, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
+                "power_w_max": max(float(r[3]) for r in rows), "samples": len(rows), "reasons": sorted(reasons)}
+
+
+def measured_peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except (OSError, ValueError):
+        return None
+
+
+# ------------------------------------------------------------ CPU oracle
+def oracle_sample(inp, n_rows: int, seed: int = 0):
+    """Time the oracle's FP8 attention (as it stands) on a bounded row sample of the workload.
+
+    The quantised inputs are prepared first (untimed); the timed part is the
+    attention of n_rows query rows x all heads over all context keys.
+    Returns (TFLOP/s, seconds, threads, description).
+    """
+    import oracle
+    N, H = inp["N"], inp["H"]
+    qs = oracle.qscale(inp["q"], N, inp["c_h"], inp["gate"])
+    s_q, s_k, s_v = (oracle.context_scales(x, N) for x in (qs, inp["k"], inp["v"]))
+    q8 = oracle.quantize(qs, s_q)
+    k8, v8 = oracle.quantize(inp["k"], s_k), oracle.quantize(inp["v"], s_v)
+    rows = np.sort(np.random.default_rng(seed).choice(inp["N"] + inp["M"], n_rows, replace=False)).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.attention(q8, k8, v8, s_q, s_k, s_v, rows=rows)
+    dt = time.perf_counter() - t0
+    fl = attn_flops(n_rows, N, H)
+    return fl / dt / 1e12, dt, oracle.num_threads(), (
+        f"oracle FP8 attention of {n_rows} sampled rows x {H} heads over all {N} context keys "
+        f"({fl:.3g} FLOP); quantisation prepared untimed")
+
+
+# ------------------------------------------------------------------ ours
+def run_ours(args):
+    import torch
+
+    import fp8_quant_logscale_b200 as sdm
+    from fp8_quant_logscale_b200 import binding
+    from fp8_quant_logscale_b200.workloads import WORKLOADS, make_inputs
+
+    rank, world = init_dist("nccl")
+    _, _, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    w = WORKLOADS[args.workload]
+    wc = WORKLOADS[CACHED_WORKLOAD]
+    inp = make_inputs(w, seed=w.seed + 1000 * rank)
+    queries_np = make_inputs(wc, seed=wc.seed + 1000 * rank, n_ctx=8, n_query=wc.n_query, heads=w.heads)["queries"]
+    B, N, M, H = inp["B"], inp["N"], inp["M"], inp["H"]
+    T = N + M
+    Mq = queries_np.shape[1]
+
+    q = torch.from_numpy(inp["q"]).to(device)
+    k = torch.from_numpy(inp["k"]).to(device)
+    v = torch.from_numpy(inp["v"]).to(device)
+    c_h = torch.from_numpy(inp["c_h"]).to(device)
+    gate = None if inp["gate"] is None else torch.from_numpy(inp["gate"]).to(device)
+    queries = torch.from_numpy(queries_np).to(device)
+    out = torch.empty_like(q)
+    pred = torch.empty_like(queries)
+    cache = sdm.FP8Cache(B, N, H, device)
+    ws_icl = sdm.new_workspace(sdm.workspace_size(binding.OP_ICL_ATTENTION, B, N, M, H, keep_cache=True), device)
+    ws_c = sdm.new_workspace(sdm.workspace_size(binding.OP_CACHED_ATTENTION, B, N, Mq, H), device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        sdm.icl_attention(q, k, v, N, c_h, gate, cache=cache, out=out, ws=ws_icl)
+        sdm.cached_attention(queries, cache, c_h, out=pred, ws=ws_c)
+
+    flops_step = attn_flops(T, N, H) + attn_flops(Mq, N, H)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    st = sdm.sync_status(ws_icl)[0] or sdm.sync_status(ws_c)[0]
+    if st:
+        raise RuntimeError(f"device error word set during warm-up: status {st}")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(device)
+    torch.cuda.synchronize(device)
+    with ClockSampler(local) as clk:
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            sdm.icl_attention(q, k, v, N, c_h, gate, cache=cache, out=out, ws=ws_icl)
+            ev[i][1].record(stream)
+            sdm.cached_attention(queries, cache, c_h, out=pred, ws=ws_c)
+            ev[i][2].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize(device)
+    barrier(device)
+    total_ms = reduce_max(start.elapsed_time(end), device)
+    icl_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    cached_us = [b.elapsed_time(c) * 1e3 for _, b, c in ev]
+    st = sdm.sync_status(ws_icl)[0] or sdm.sync_status(ws_c)[0]
+    if st:
+        raise RuntimeError(f"device error word set during timing: status {st}")
+
+    # The dominant kernel alone (FP8 attention of all T rows over the same
+    # cache), timed with CUDA events on the launching stream.
+    kern_ms = []
+    q8_rows, _ = sdm.fp8_quantize_context(sdm.qscale_fused(q, c_h, N, gate), k, v, N, cache=cache)
+    ws_a = sdm.new_workspace(256, device)
+    for i in range(args.warmup + args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        sdm.fp8_attention(q8_rows, cache, split=False, out=out, ws=ws_a)
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        if i >= args.warmup:
+            kern_ms.append(a.elapsed_time(b))
+    del q8_rows
+
+    # End to end through the public API with host buffers: pinned H2D of the
+    # step's inputs, both calls, D2H of both outputs, every step.
+    e2e = None
+    if not args.skip_e2e:
+        hq, hk, hv = (torch.from_numpy(a).pin_memory() for a in (inp["q"], inp["k"], inp["v"]))
+        hqq = torch.from_numpy(queries_np).pin_memory()
+        hout, hpred = torch.empty_like(hq).pin_memory(), torch.empty_like(hqq).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hqq))
+        d2h = hout.numel() * 2 + hpred.numel() * 2
+        e_steps = max(1, min(args.steps, 3))
+        barrier(device)
+        torch.cuda.synchronize(device)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e_steps):
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            queries.copy_(hqq, non_blocking=True)
+            sdm.icl_attention(q, k, v, N, c_h, gate, cache=cache, out=out, ws=ws_icl)
+            sdm.cached_attention(queries, cache, c_h, out=pred, ws=ws_c)
+            hout.copy_(out, non_blocking=True)
+            hpred.copy_(pred, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        e_ms = reduce_max(a.elapsed_time(b) / e_steps, device)
+        e2e = {"value": world * flops_step / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e_ms,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    ms_per_step = total_ms / args.steps
+    value = world * flops_step / (ms_per_step * 1e-3) / 1e12
+    peaks = measured_peaks()
+    if peaks:
+        fp8_peak = peaks["bf16_tflops_sustained"] * FP8_NOMINAL_TFLOPS / BF16_NOMINAL_TFLOPS
+        peak_src = "of measured (bf16 sustained x nominal fp8/bf16 ratio 2)"
+    else:
+        fp8_peak = 1400.0 * 2
+        peak_src = "of fallback (1.4 PF bf16 sustained x 2)"
+    kmean = statistics.mean(kern_ms)
+    achieved = attn_flops(T, N, H) / (kmean * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8_e4m3", "data": "synthetic (seeded N(0,1) fp16, per-rank seed)",
+        "config": {"workload": f"{w.name} fit + {wc.name} predict", "batch": B, "n_ctx": N, "n_query": M,
+                   "predict_queries": Mq, "heads": H, "head_dim": 64,
+                   "l2": "inputs exceed L2 (q,k,v 1.6 GB; FP8 cache 0.54 GB): no flush needed",
+                   "parallelism": f"replicas x{world} (independent problems)" if world > 1 else "single GPU"},
+        "icl_ms": statistics.median(icl_ms), "cached_us": statistics.median(cached_us),
+        "attention_kernel_ms": kmean,
+        "pct_fp8_peak": 100.0 * achieved / fp8_peak, "pct_fp8_nominal": 100.0 * achieved / FP8_NOMINAL_TFLOPS,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
+                     "frac": achieved / fp8_peak, "traffic": args.traffic, "peak_source": peak_src,
+                     "kernel": "icl_attention_kernel (FP8 attention of all rows)"},
+        "gpu_launches": args.steps * 9,
+        "clocks": clk.summary(),
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        val, dt, cores, desc = oracle_sample(inp, args.cpu_rows)
+        line["cpu_baseline"] = {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                "sample": desc, "seconds": dt}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------- reference
+def run_reference(args):
+    """The oracle as it stands, on the host cores: rank 0 only, bounded row samples."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    from fp8_quant_logscale_b200.workloads import WORKLOADS, make_inputs
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w)
+    N, H = inp["N"], inp["H"]
+    qs = oracle.qscale(inp["q"], N, inp["c_h"], inp["gate"])
+    s_q, s_k, s_v = (oracle.context_scales(x, N) for x in (qs, inp["k"], inp["v"]))
+    q8 = oracle.quantize(qs, s_q)
+    k8, v8 = oracle.quantize(inp["k"], s_k), oracle.quantize(inp["v"], s_v)
+    rng = np.random.default_rng(0)
+    times = []
+    for i in range(args.warmup + args.steps):
+        rows = np.sort(rng.choice(N + inp["M"], args.cpu_rows, replace=False)).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.attention(q8, k8, v8, s_q, s_k, s_v, rows=rows)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    dt = statistics.mean(times)
+    fl = attn_flops(args.cpu_rows, N, H)
+    val = fl / dt / 1e12
+    sample = (f"each step: oracle FP8 attention of {args.cpu_rows} sampled rows x {H} heads over all {N} "
+              f"context keys of {w.name}; quantisation prepared once, untimed")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3", "data": "synthetic",
+        "config": {"workload": w.name, "n_ctx": N, "n_query": inp["M"], "heads": H, "head_dim": 64,
+                   "parallelism": "host cores (OpenMP)"},
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, help="workload name (profiling runs use smaller ones)")
+    ap.add_argument("--cpu-rows", type=int, default=64, help="rows of the oracle's timed sample")
+    ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per attention launch from an ncu capture of the current kernel")
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -273,6 +273,7 @@ sdm_status sdm_fp8_attention(const uint8_t* q8, int32_t B, int64_t rows, const s
   a.N = cache->n_ctx;
   a.ld_v = cache->ld_v;
   a.scales = cache->scales;
+  a.partial = split != 0;
   a.n_splits = split ? n_splits_for(cache->n_ctx) : 1;
   a.split_keys = kSplitKeys;
   a.out = reinterpret_cast<__half*>(out);
@@ -336,6 +337,7 @@ sdm_status sdm_icl_attention(const void* q, const void* k, const void* v, int32_
   a.N = N;
   a.ld_v = c->ld_v;
   a.scales = c->scales;
+  a.partial = false;
   a.n_splits = 1;
   a.split_keys = kSplitKeys;
   a.out = reinterpret_cast<__half*>(out);
@@ -379,6 +381,7 @@ sdm_status sdm_cached_attention(const void* q, int32_t B, int64_t M, int32_t H, 
   a.N = N;
   a.ld_v = cache->ld_v;
   a.scales = cache->scales;
+  a.partial = true;
   a.n_splits = n_splits_for(N);
   a.split_keys = kSplitKeys;
   a.out = reinterpret_cast<__half*>(out);

@@ -72,6 +72,7 @@ struct KParams {
   int32_t BH, H;
   int64_t T, N;
   int64_t n_pairs, n_splits, split_keys;
+  int32_t partial;
   const float* scales;  // [3][BH]
   __half* out;
   float* part_acc;
@@ -112,8 +113,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t split = rest % p.n_splits;
   const int64_t bh = rest / p.n_splits;
   const int64_t row0 = pair * (kTiles * kQTile);
-  const int64_t kv_begin = (p.n_splits > 1) ? split * p.split_keys : 0;
-  const int64_t kv_end = (p.n_splits > 1) ? min(p.N, kv_begin + p.split_keys) : p.N;
+  const int64_t kv_begin = p.partial ? split * p.split_keys : 0;
+  const int64_t kv_end = p.partial ? min(p.N, kv_begin + p.split_keys) : p.N;
   const int n_tiles = static_cast<int>((kv_end - kv_begin + kKvTile - 1) / kKvTile);
 
   // ---- set-up
@@ -345,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t row = row0 + (int64_t)t * kQTile + 32 * wq + lane;
       if (row < p.T) {
         const float lf = __uint_as_float(l);
-        if (p.n_splits == 1) {
+        if (!p.partial) {
           const int64_t b = bh / p.H, h = bh % p.H;
           uint4* dst = reinterpret_cast<uint4*>(p.out + ((b * p.T + row) * p.H + h) * kHeadDim);
 #pragma unroll
@@ -469,8 +470,9 @@ cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t
   p.T = a.T;
   p.N = a.N;
   p.n_pairs = (a.T + kTiles * kQTile - 1) / (kTiles * kQTile);
-  p.n_splits = a.n_splits;
+  p.n_splits = a.partial ? a.n_splits : 1;
   p.split_keys = a.split_keys;
+  p.partial = a.partial ? 1 : 0;
   p.scales = a.scales;
   p.out = a.out;
   p.part_acc = a.part_acc;

@@ -54,8 +54,9 @@ struct AttnArgs {
   int64_t N;           // context keys
   int64_t ld_v;        // V8 transposed row length (keys), multiple of 128
   const float* scales; // [3][B][H]: s_q, s_k, s_v
-  int64_t n_splits;    // 1: single pass, final output; >1: split-KV partials
-  int64_t split_keys;  // keys per split (multiple of kKvTile) when n_splits > 1
+  bool partial;        // false: one pass, normalised fp16 output; true: split-KV partials
+  int64_t n_splits;    // number of key chunks (1 when !partial)
+  int64_t split_keys;  // keys per chunk (multiple of kKvTile) when partial
   __half* out;         // final: [B][T][H][64] fp16
   float* part_acc;     // split: [S][B*H][T][64]
   float* part_ml;      // split: [S][B*H][T][2] (m2, l)

@@ -88,6 +88,7 @@ uint8_t orc_e4m3_encode(double y) {
     uint8_t sign = signbit(y) ? 0x80 : 0;
     double a = fabs(y);
     if (a >= 448.0) return sign | 0x7E;
+    if (a <= 0x1p-10) return sign;             /* at or below half of 2^-9: ties to even 0 */
     int e;                                     /* binade: a in [2^e, 2^(e+1)) */
     if (a < 0x1p-6) e = -6;                    /* subnormals share the 2^-6 spacing */
     else { int E; frexp(a, &E); e = E - 1; }

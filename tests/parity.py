@@ -21,11 +21,20 @@ def host(t):
     return t.detach().cpu().numpy()
 
 
+def fp16_ulp(x):
+    """Spacing of fp16 values at |x| (2^-24 in the subnormal range)."""
+    a = np.abs(np.asarray(x, np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -14)))
+    return np.exp2(e - 10)
+
+
 def gate(gpu_out, ref_out, allow, what=""):
-    """Assert |gpu - oracle| <= MAX_ABS + allowance elementwise and mean |.| <= MEAN_ABS."""
+    """Assert |gpu - oracle| <= max(MAX_ABS, 1 fp16 ulp of the value) + allowance
+    elementwise, and mean |gpu - oracle| <= MEAN_ABS.  The output is fp16, so
+    where one ulp exceeds MAX_ABS (|O| >= 64) rounding alone may take one ulp."""
     g = host(gpu_out).astype(np.float64) if isinstance(gpu_out, torch.Tensor) else gpu_out.astype(np.float64)
     d = np.abs(g - ref_out)
-    excess = d - allow
+    excess = d - allow - np.maximum(0.0, fp16_ulp(ref_out) - MAX_ABS)
     strict = allow == 0
     stats = dict(max_abs=float(d.max()), mean_abs=float(d.mean()),
                  max_abs_strict=float(d[strict].max()) if strict.any() else 0.0,
