@@ -26,6 +26,7 @@
 // TMEM (512 columns): S0 [0,128)  S1 [128,256)  O0 [256,336)  O1 [336,416).
 #include <math.h>
 
+#include "exp2_poly.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -93,6 +94,79 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint3
       atomicOr(err, kErrTimeoutDrain);
       return;
     }
+  }
+}
+
+// Keys at or past `nvalid` (counted from the tile start) get logit -inf, so
+// they neither raise the max nor receive probability.
+__device__ __forceinline__ void mask_keys(uint32_t (&ra)[32], uint32_t (&rb)[32], int col0, int64_t nvalid) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    if (col0 + i >= nvalid) ra[i] = __float_as_uint(-INFINITY);
+    if (col0 + 32 + i >= nvalid) rb[i] = __float_as_uint(-INFINITY);
+  }
+}
+
+// 2^t on the FMA pipe for a pair of lanes: t = j + f with j = round(t) (the
+// 1.5*2^23 rounding trick), f in [-1/2, 1/2], 2^f from the degree-4 Remez
+// polynomial of exp2_poly.cuh (relative error < 3e-6), and 2^j added to the
+// exponent field.  t is clamped at -30 first: every result below 2^-10 is an
+// e4m3 zero anyway, and the clamp keeps the exponent arithmetic in range.
+__device__ __forceinline__ void exp2_fma2(float t0, float t1, float& p0, float& p1) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  t0 = fmaxf(t0, -30.0f);
+  t1 = fmaxf(t1, -30.0f);
+  float r0, r1, j0, j1, f0, f1;
+  add2(r0, r1, t0, t1, kRound, kRound);
+  sub2(j0, j1, r0, r1, kRound, kRound);
+  sub2(f0, f1, t0, t1, j0, j1);
+  float q0 = kExp2C4, q1 = kExp2C4;
+  fma2(q0, q1, q0, q1, f0, f1, kExp2C3, kExp2C3);
+  fma2(q0, q1, q0, q1, f0, f1, kExp2C2, kExp2C2);
+  fma2(q0, q1, q0, q1, f0, f1, kExp2C1, kExp2C1);
+  fma2(q0, q1, q0, q1, f0, f1, kExp2C0, kExp2C0);
+  // the bit pattern of r holds j + 1.5*2^23; shifted by 23 the constant part
+  // vanishes modulo 2^32, leaving j in the exponent field
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(r0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(r1) << 23));
+}
+
+// Which of the 8 four-key words of a 32-key chunk take the FMA-pipe 2^x:
+// kPolyEighths of them, spread evenly; the others use the MUFU ex2.
+#ifndef SDM_POLY_EIGHTHS
+#define SDM_POLY_EIGHTHS 2
+#endif
+constexpr int kPolyEighths = SDM_POLY_EIGHTHS;
+__host__ __device__ constexpr bool poly_word(int w) {
+  return (w * kPolyEighths) / 8 != ((w + 1) * kPolyEighths) / 8;
+}
+
+// Four logits -> one 32-bit column of four e4m3 probabilities (key 4w+i in byte i).
+template <bool kPoly>
+__device__ __forceinline__ uint32_t p_word(const uint32_t* z, float c2, float nm2) {
+  float t0, t1, t2, t3, p0, p1, p2, p3;
+  fma2(t0, t1, __uint_as_float(z[0]), __uint_as_float(z[1]), c2, c2, nm2, nm2);
+  fma2(t2, t3, __uint_as_float(z[2]), __uint_as_float(z[3]), c2, c2, nm2, nm2);
+  if (kPoly) {
+    exp2_fma2(t0, t1, p0, p1);
+    exp2_fma2(t2, t3, p2, p3);
+  } else {
+    p0 = ex2_approx(t0);
+    p1 = ex2_approx(t1);
+    p2 = ex2_approx(t2);
+    p3 = ex2_approx(t3);
+  }
+  return e4m3x2(p0, p1) | (e4m3x2(p2, p3) << 16);
+}
+
+// Words W..7 of two 32-key chunks (compile-time word index selects the 2^x path).
+template <int W>
+__device__ __forceinline__ void p_words(const uint32_t (&ra)[32], const uint32_t (&rb)[32], uint32_t (&pw)[16],
+                                        float c2, float nm2) {
+  if constexpr (W < 8) {
+    pw[W] = p_word<poly_word(W)>(ra + 4 * W, c2, nm2);
+    pw[8 + W] = p_word<poly_word(W)>(rb + 4 * W, c2, nm2);
+    p_words<W + 1>(ra, rb, pw, c2, nm2);
   }
 }
 
@@ -274,23 +348,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      uint32_t r[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(t_s + 32 * c, r[c]);
-      tmem_ld_wait();
       const int64_t nvalid = kv_end - (kv_begin + (int64_t)it * kKvTile);
-      if (nvalid < kKvTile) {
+      const bool ragged = nvalid < kKvTile;
+      // pass 1: the tile's row max, 64 logits in registers at a time
+      float mx0 = m_run, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+      for (int h = 0; h < 2; ++h) {
+        uint32_t ra[32], rb[32];
+        tmem_ld_32x32b_x32(t_s + 64 * h, ra);
+        tmem_ld_32x32b_x32(t_s + 64 * h + 32, rb);
+        tmem_ld_wait();
+        if (ragged) mask_keys(ra, rb, 64 * h, nvalid);
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (32 * c + i >= nvalid) r[c][i] = __float_as_uint(-INFINITY);
+        for (int i = 0; i < 32; i += 4) {
+          mx0 = max3(mx0, __uint_as_float(ra[i + 0]), __uint_as_float(rb[i + 0]));
+          mx1 = max3(mx1, __uint_as_float(ra[i + 1]), __uint_as_float(rb[i + 1]));
+          mx2 = max3(mx2, __uint_as_float(ra[i + 2]), __uint_as_float(rb[i + 2]));
+          mx3 = max3(mx3, __uint_as_float(ra[i + 3]), __uint_as_float(rb[i + 3]));
+        }
       }
-      float mt = m_run;
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) mt = fmaxf(mt, __uint_as_float(r[c][i]));
+      const float mt = max3(mx0, mx1, fmaxf(mx2, mx3));
       const bool up = mt > m_run;
       const float m2_new = up ? __fmul_rn(mt, c2) : m2;
       if (it > 0 && __any_sync(0xffffffffu, up)) {
@@ -312,19 +389,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       m_run = mt;
       m2 = m2_new;
-      // P = 2^(fma(z, c2, -m2)) in (0, 1], four e4m3 codes per 32-bit column
-      uint32_t pw[32];
+      // pass 2: P = 2^(fma(z, c2, -m2)) in (0, 1] -> e4m3, four codes per
+      // 32-bit TMEM column, written over S columns that are already consumed
+      const float nm2 = -m2;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-          const float p0 = ex2_approx(__fmaf_rn(__uint_as_float(r[c][4 * w + 0]), c2, -m2));
-          const float p1 = ex2_approx(__fmaf_rn(__uint_as_float(r[c][4 * w + 1]), c2, -m2));
-          const float p2 = ex2_approx(__fmaf_rn(__uint_as_float(r[c][4 * w + 2]), c2, -m2));
-          const float p3 = ex2_approx(__fmaf_rn(__uint_as_float(r[c][4 * w + 3]), c2, -m2));
-          pw[8 * c + w] = e4m3x2(p0, p1) | (e4m3x2(p2, p3) << 16);
-        }
-      tmem_st_32x32b_x32(t_s, pw);
+      for (int h = 0; h < 2; ++h) {
+        uint32_t ra[32], rb[32];
+        tmem_ld_32x32b_x32(t_s + 64 * h, ra);
+        tmem_ld_32x32b_x32(t_s + 64 * h + 32, rb);
+        tmem_ld_wait();
+        if (ragged) mask_keys(ra, rb, 64 * h, nvalid);
+        uint32_t pw[16];
+        p_words<0>(ra, rb, pw, c2, nm2);
+        tmem_st_32x32b_x16(t_s + 16 * h, pw);
+      }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();

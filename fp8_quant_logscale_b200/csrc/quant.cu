@@ -16,6 +16,8 @@
 namespace sdm {
 namespace {
 
+constexpr int kUnroll = 4;  // 16-byte loads in flight per thread
+
 __device__ __forceinline__ float head_scale(const QScale& qs, int h) {
   // s_h = fp16(c_h * lam): fp32 product, one rounding to the query dtype.
   return __half2float(__float2half_rn(__fmul_rn(__ldg(qs.c_h + h), qs.lam)));
@@ -68,22 +70,31 @@ inline int num_sms() {
 __global__ void __launch_bounds__(256) qscale_kernel(const __half* __restrict__ q, __half* __restrict__ out,
                                                      int64_t n_vec, int H, QScale qs) {
   const bool gated = qs.gate != nullptr;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_vec; i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t seg = i >> 3;  // (b*rows + r)*H + h
-    const int h = static_cast<int>(seg % H);
-    const int64_t br = seg / H;
-    const float s = head_scale(qs, h);
-    const float w = gated ? gate_factor(qs, br, H, h) : 1.0f;
-    const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(q) + i);
-    float f[8];
-    unpack8(raw, f);
-    uint4 res;
-    __half2* r2 = reinterpret_cast<__half2*>(&res);
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i0 < n_vec; i0 += kUnroll * stride) {
+    uint4 raw[kUnroll];
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-      r2[k] = __halves2half2(__float2half_rn(qscale1(f[2 * k], s, gated, w)),
-                             __float2half_rn(qscale1(f[2 * k + 1], s, gated, w)));
-    __stcs(reinterpret_cast<uint4*>(out) + i, res);
+    for (int u = 0; u < kUnroll; ++u)  // all loads first: kUnroll 16-byte requests in flight
+      if (i0 + u * stride < n_vec) raw[u] = __ldcs(reinterpret_cast<const uint4*>(q) + i0 + u * stride);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i >= n_vec) break;
+      const int64_t seg = i >> 3;  // (b*rows + r)*H + h
+      const int h = static_cast<int>(seg % H);
+      const int64_t br = seg / H;
+      const float s = head_scale(qs, h);
+      const float w = gated ? gate_factor(qs, br, H, h) : 1.0f;
+      float f[8];
+      unpack8(raw[u], f);
+      uint4 res;
+      __half2* r2 = reinterpret_cast<__half2*>(&res);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        r2[k] = __halves2half2(__float2half_rn(qscale1(f[2 * k], s, gated, w)),
+                               __float2half_rn(qscale1(f[2 * k + 1], s, gated, w)));
+      __stcs(reinterpret_cast<uint4*>(out) + i, res);
+    }
   }
 }
 
@@ -110,14 +121,23 @@ __global__ void context_amax_kernel(RowsDesc q, QScale qs, RowsDesc k, RowsDesc 
 
   const float s = do_q ? head_scale(qs, h) : 1.0f;
   float m = 0.0f;
-  for (int64_t r = r0 + t / vecs_per_row; r < r1; r += row_step) {
-    const int64_t br = (int64_t)b * X.rows + r;
-    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(X.x + br * H * kHeadDim) + vrow);
-    const float w = gated ? gate_factor(qs, br, H, h) : 1.0f;
-    float f[8];
-    unpack8(raw, f);
+  for (int64_t r = r0 + t / vecs_per_row; r < r1; r += kUnroll * row_step) {
+    uint4 raw[kUnroll];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(do_q ? qscale1(f[e], s, gated, w) : f[e]));
+    for (int u = 0; u < kUnroll; ++u)  // all loads first: kUnroll 16-byte requests in flight
+      if (r + u * row_step < r1)
+        raw[u] = __ldg(reinterpret_cast<const uint4*>(X.x + ((int64_t)b * X.rows + r + u * row_step) * H * kHeadDim) +
+                       vrow);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      if (r + u * row_step >= r1) break;
+      const int64_t br = (int64_t)b * X.rows + r + u * row_step;
+      const float w = gated ? gate_factor(qs, br, H, h) : 1.0f;
+      float f[8];
+      unpack8(raw[u], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(do_q ? qscale1(f[e], s, gated, w) : f[e]));
+    }
   }
   // reduce over the 8 lanes of the (row, head) segment, then per head in smem
   const unsigned group = 0xFFu << (threadIdx.x & 24);
@@ -156,18 +176,27 @@ __global__ void quantize_rows_kernel(RowsDesc X, QScale qs, int64_t n_rows, cons
   const float s = do_q ? head_scale(qs, h) : 1.0f;
   const float sx = __ldg(scale + b * H + h);
   uint8_t* dbase = dst + ((int64_t)b * H + h) * dst_rows * kHeadDim + j * 8;
-  for (int64_t r = r0 + t / vecs_per_row; r < r1; r += row_step) {
-    const int64_t br = (int64_t)b * X.rows + r;
-    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(X.x + br * H * kHeadDim) + vrow);
-    const float w = gated ? gate_factor(qs, br, H, h) : 1.0f;
-    float f[8];
-    unpack8(raw, f);
+  for (int64_t r = r0 + t / vecs_per_row; r < r1; r += kUnroll * row_step) {
+    uint4 raw[kUnroll];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) f[e] = __fdiv_rn(do_q ? qscale1(f[e], s, gated, w) : f[e], sx);
-    uint2 codes;
-    codes.x = e4m3x2(f[0], f[1]) | (e4m3x2(f[2], f[3]) << 16);
-    codes.y = e4m3x2(f[4], f[5]) | (e4m3x2(f[6], f[7]) << 16);
-    *reinterpret_cast<uint2*>(dbase + r * kHeadDim) = codes;
+    for (int u = 0; u < kUnroll; ++u)  // all loads first: kUnroll 16-byte requests in flight
+      if (r + u * row_step < r1)
+        raw[u] = __ldcs(reinterpret_cast<const uint4*>(X.x + ((int64_t)b * X.rows + r + u * row_step) * H * kHeadDim) +
+                        vrow);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t rr = r + u * row_step;
+      if (rr >= r1) break;
+      const float w = gated ? gate_factor(qs, (int64_t)b * X.rows + rr, H, h) : 1.0f;
+      float f[8];
+      unpack8(raw[u], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = __fdiv_rn(do_q ? qscale1(f[e], s, gated, w) : f[e], sx);
+      uint2 codes;
+      codes.x = e4m3x2(f[0], f[1]) | (e4m3x2(f[2], f[3]) << 16);
+      codes.y = e4m3x2(f[4], f[5]) | (e4m3x2(f[6], f[7]) << 16);
+      *reinterpret_cast<uint2*>(dbase + rr * kHeadDim) = codes;
+    }
   }
 }
 
@@ -185,16 +214,21 @@ __global__ void __launch_bounds__(256) quantize_vt_kernel(RowsDesc V, int64_t n_
   const int t = threadIdx.x;
   const int j = t & 7;  // elements 8j..8j+7
   uint8_t* tb = reinterpret_cast<uint8_t*>(&tile[0][0]);
+  uint4 raws[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {  // all loads first: four 16-byte requests in flight
+    const int64_t r = r0 + (t >> 3) + 32 * i;
+    if (r < n_ctx)
+      raws[i] = __ldcs(reinterpret_cast<const uint4*>(V.x + (((int64_t)b * V.rows + r) * H + h) * kHeadDim) + j);
+  }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int rl = (t >> 3) + 32 * i;
     const int64_t r = r0 + rl;
     uint32_t lo = 0, hi = 0;
     if (r < n_ctx) {
-      const uint4 raw =
-          __ldg(reinterpret_cast<const uint4*>(V.x + (((int64_t)b * V.rows + r) * H + h) * kHeadDim) + j);
       float f[8];
-      unpack8(raw, f);
+      unpack8(raws[i], f);
 #pragma unroll
       for (int e = 0; e < 8; ++e) f[e] = __fdiv_rn(f[e], sx);
       lo = e4m3x2(f[0], f[1]) | (e4m3x2(f[2], f[3]) << 16);
@@ -226,7 +260,7 @@ cudaError_t launch_qscale(const __half* q, __half* out, int32_t B, int64_t rows,
                           cudaStream_t st) {
   const int64_t n_vec = (int64_t)B * rows * H * (kHeadDim / 8);
   if (n_vec == 0) return cudaSuccess;
-  const int64_t want = (n_vec + 255) / 256;
+  const int64_t want = (n_vec + 256 * kUnroll - 1) / (256 * kUnroll);
   const int grid = static_cast<int>(want < (int64_t)num_sms() * 8 ? want : (int64_t)num_sms() * 8);
   qscale_kernel<<<grid, 256, 0, st>>>(q, out, n_vec, H, qs);
   return cudaGetLastError();
@@ -236,8 +270,8 @@ cudaError_t launch_context_amax(RowsDesc q, QScale qs, RowsDesc k, RowsDesc v, i
                                 cudaStream_t st) {
   const int threads = row_threads(q.H);
   const int rows_per_pass = threads / (8 * q.H);
-  // about 4 CTAs per SM over the three tensors
-  int64_t chunks = ((int64_t)num_sms() * 4 + 3 * q.B - 1) / (3 * q.B);
+  // about 8 CTAs per SM over the three tensors
+  int64_t chunks = ((int64_t)num_sms() * 8 + 3 * q.B - 1) / (3 * q.B);
   int64_t rows_per_cta = (n_ctx + chunks - 1) / chunks;
   rows_per_cta = ((rows_per_cta + rows_per_pass - 1) / rows_per_pass) * rows_per_pass;
   chunks = (n_ctx + rows_per_cta - 1) / rows_per_cta;
@@ -257,7 +291,7 @@ cudaError_t launch_quantize_rows(RowsDesc x, QScale qs, int64_t n_rows, const fl
   if (n_rows == 0) return cudaSuccess;
   const int threads = row_threads(x.H);
   const int rows_per_pass = threads / (8 * x.H);
-  int64_t chunks = ((int64_t)num_sms() * 4 + x.B - 1) / x.B;
+  int64_t chunks = ((int64_t)num_sms() * 8 + x.B - 1) / x.B;
   int64_t rows_per_cta = (n_rows + chunks - 1) / chunks;
   rows_per_cta = ((rows_per_cta + rows_per_pass - 1) / rows_per_pass) * rows_per_pass;
   chunks = (n_rows + rows_per_cta - 1) / rows_per_cta;
