@@ -25,8 +25,9 @@ HEAD_DIM = 64
 
 # Every symbol the header declares (checked by the ABI tests).
 EXPORTS = ("sdm_status_string", "sdm_version", "sdm_cache_layout", "sdm_workspace_size", "sdm_qscale_fused",
-           "sdm_fp8_quantize_context", "sdm_fp8_attention", "sdm_icl_attention", "sdm_cached_attention",
-           "sdm_sync_status")
+           "sdm_fp8_quantize_context", "sdm_fp8_quantize_context_noalloc", "sdm_fp8_attention", "sdm_icl_attention",
+           "sdm_cached_attention", "sdm_sync_status")
+NOALLOC_MAX_BATCH_HEADS = 4096
 
 
 class SdmError(RuntimeError):
@@ -68,6 +69,9 @@ def lib() -> ctypes.CDLL:
         L.sdm_fp8_quantize_context.restype = ctypes.c_int
         L.sdm_fp8_quantize_context.argtypes = [_P, _P, _P, _I32, _I64, _I64, _I32, _I32, _P,
                                                ctypes.POINTER(CacheStruct), _P, _SZ, _P]
+        L.sdm_fp8_quantize_context_noalloc.restype = ctypes.c_int
+        L.sdm_fp8_quantize_context_noalloc.argtypes = [_P, _P, _P, _I32, _I64, _I64, _I32, _I32, _P,
+                                                       ctypes.POINTER(CacheStruct), _P]
         L.sdm_fp8_attention.restype = ctypes.c_int
         L.sdm_fp8_attention.argtypes = [_P, _I32, _I64, ctypes.POINTER(CacheStruct), _P, _I32, _P, _SZ, _P]
         L.sdm_icl_attention.restype = ctypes.c_int
@@ -191,6 +195,25 @@ def fp8_quantize_context(q_scaled: torch.Tensor, k: torch.Tensor, v: torch.Tenso
         _check(lib().sdm_fp8_quantize_context(_ptr(q_scaled), _ptr(k), _ptr(v), B, n_ctx, M, H, d, _ptr(q8),
                                               ctypes.byref(cache.struct), _ptr(ws), ws.numel(), _stream(dev)),
                "sdm_fp8_quantize_context")
+    return q8, cache
+
+
+def fp8_quantize_context_noalloc(q_scaled: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_ctx: int,
+                                 cache: FP8Cache | None = None, q8: torch.Tensor | None = None):
+    """fp8_quantize_context for callers that cannot provide a workspace: the
+    library keeps the amax scratch in a fixed device array of its own (B*H up
+    to NOALLOC_MAX_BATCH_HEADS; calls that overlap on the GPU race on it)."""
+    _want(q_scaled, torch.float16, "q_scaled", 4)
+    _want(k, torch.float16, "k", 4)
+    _want(v, torch.float16, "v", 4)
+    B, T, H, d = q_scaled.shape
+    dev = q_scaled.device
+    cache = FP8Cache(B, n_ctx, H, dev) if cache is None else cache
+    q8 = torch.empty((B, H, T, d), dtype=torch.uint8, device=dev) if q8 is None else q8
+    with torch.cuda.device(dev):
+        _check(lib().sdm_fp8_quantize_context_noalloc(_ptr(q_scaled), _ptr(k), _ptr(v), B, n_ctx, T - n_ctx, H, d,
+                                                      _ptr(q8), ctypes.byref(cache.struct), _stream(dev)),
+               "sdm_fp8_quantize_context_noalloc")
     return q8, cache
 
 

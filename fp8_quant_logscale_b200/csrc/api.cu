@@ -5,6 +5,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "../../include/sdm_fp8.h"
 #include "kernels.cuh"
 
@@ -414,3 +416,76 @@ sdm_status sdm_sync_status(void* ws, void* stream, uint32_t* flags) {
 }
 
 }  // extern "C"
+// ---------------------------------------------------------------------------
+// Context quantisation for callers that cannot provide a workspace.
+//
+// Some callers of this library cannot allocate device memory for it: code on a
+// latency-critical path that must not call cudaMalloc (which can synchronise
+// the whole device), plugins whose host framework owns all device memory
+// behind its own allocator, and hooks that run where no allocation API is
+// reachable.  The only scratch the quantisation step needs is its per-(tensor,
+// batch, head) amax accumulator, so this variant keeps it in a fixed
+// file-scope device array instead of the caller's workspace.  The array is
+// part of the library image: every GPU that loads the library holds it
+// (48 KiB) until the process exits.
+namespace {
+
+constexpr int kNoAllocMaxBatchHeads = SDM_NOALLOC_MAX_BATCH_HEADS;
+static __device__ __align__(256) uint32_t g_noalloc_amax[3 * kNoAllocMaxBatchHeads];
+
+// In host code `g_noalloc_amax` names a host-side stand-in, not device memory,
+// so kernels must be given the address the runtime reports for it -- looked up
+// once per device, with that device current.
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+uint32_t* g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+sdm_status noalloc_scratch(int dev, uint32_t** out) {
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return SDM_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_amax) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return SDM_ERR_CUDA;
+    }
+    g_noalloc_addr[dev] = static_cast<uint32_t*>(p);
+  }
+  *out = g_noalloc_addr[dev];
+  return SDM_OK;
+}
+
+}  // namespace
+
+extern "C" sdm_status sdm_fp8_quantize_context_noalloc(const void* q_scaled, const void* k, const void* v,
+                                                       int32_t B, int64_t N, int64_t M, int32_t H, int32_t d,
+                                                       uint8_t* q8, sdm_fp8_cache* cache, void* stream) {
+  SDM_TRY(check_shape(B, N, M, H, d));
+  if (N < 1) return SDM_ERR_INVALID_ARG;
+  if ((int64_t)B * H > kNoAllocMaxBatchHeads) return SDM_ERR_UNSUPPORTED;
+  const int dev = current_device();
+  if (dev < 0) return SDM_ERR_CUDA;
+  SDM_TRY(check_tensor(q_scaled, dev));
+  SDM_TRY(check_tensor(k, dev));
+  SDM_TRY(check_tensor(v, dev));
+  SDM_TRY(check_tensor(q8, dev));
+  SDM_TRY(check_cache(cache, B, H, d, dev, false));
+  if (cache->n_ctx != N) return SDM_ERR_CACHE_MISMATCH;
+  uint32_t* amax = nullptr;
+  SDM_TRY(noalloc_scratch(dev, &amax));
+  cudaStream_t st = as_stream(stream);
+  const int64_t T = N + M;
+  const int64_t BH = (int64_t)B * H;
+  // the array keeps whatever the previous call left: the max accumulators restart at zero
+  SDM_CUDA(cudaMemsetAsync(amax, 0, 3 * (size_t)BH * sizeof(uint32_t), st));
+  RowsDesc dq{reinterpret_cast<const __half*>(q_scaled), B, H, T};
+  RowsDesc dk{reinterpret_cast<const __half*>(k), B, H, N};
+  RowsDesc dv{reinterpret_cast<const __half*>(v), B, H, N};
+  SDM_CUDA(launch_context_amax(dq, no_qscale(), dk, dv, N, amax, st));
+  SDM_CUDA(launch_scales_from_amax(amax, B * H, cache->scales, st));
+  SDM_CUDA(launch_quantize_rows(dq, no_qscale(), T, cache->scales, q8, T, st));
+  SDM_CUDA(launch_quantize_rows(dk, no_qscale(), N, cache->scales + BH, cache->k8, N, st));
+  SDM_CUDA(launch_quantize_vt(dv, N, cache->scales + 2 * BH, cache->v8t, cache->ld_v, st));
+  cache->filled = 1;
+  return SDM_OK;
+}

@@ -203,6 +203,29 @@ sdm_status sdm_cached_attention(const void* q, int32_t batch, int64_t n_query, i
                                 size_t ws_bytes, void* stream);
 
 /*
+ * Step 2 without a workspace.  This entry point has no counterpart in the
+ * pages: it exists for callers that cannot allocate device memory for the
+ * library -- code that must not call cudaMalloc on its path (cudaMalloc can
+ * synchronise the device), plugins whose framework owns all device memory, and
+ * hooks with no allocation API at hand.  Same arguments, layouts, results and
+ * errors as sdm_fp8_quantize_context, minus ws/ws_bytes.
+ *   - Its scratch (the amax accumulators, 3*B*H words) is a fixed array inside
+ *     the library image, sized for B*H <= SDM_NOALLOC_MAX_BATCH_HEADS (48 KiB);
+ *     every GPU that loads the library holds it until the process exits.
+ *     Larger B*H returns SDM_ERR_UNSUPPORTED before any work is enqueued.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - The call allocates nothing and clears the scratch it uses on `stream`.
+ *   - All calls share the one array: calls that overlap on the GPU (another
+ *     stream, another thread) race on it and may produce wrong scales.  Order
+ *     them on one stream or synchronise between them.
+ */
+#define SDM_NOALLOC_MAX_BATCH_HEADS 4096
+sdm_status sdm_fp8_quantize_context_noalloc(const void* q_scaled, const void* k, const void* v, int32_t batch,
+                                            int64_t n_ctx, int64_t n_query, int32_t heads, int32_t head_dim,
+                                            uint8_t* q8, sdm_fp8_cache* cache, void* stream);
+
+/*
  * Wait for `stream`, then read and clear the device error word at the head of
  * a workspace used by the calls above.  Returns SDM_OK, SDM_ERR_TIMEOUT (an
  * in-kernel wait gave up; `*flags` gets the raw bits if flags != NULL) or
