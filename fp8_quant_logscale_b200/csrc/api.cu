@@ -76,7 +76,7 @@ sdm_status check_tensor(const void* p, int dev) {
 
 // Workspace carve-up.  Offsets are 1 KB aligned; the error word sits at 0.
 struct WsLayout {
-  size_t amax = 0, q8 = 0, k8 = 0, v8t = 0, scales = 0, part_acc = 0, part_ml = 0, total = 0;
+  size_t amax = 0, gate_w = 0, q8 = 0, k8 = 0, v8t = 0, scales = 0, part_acc = 0, part_ml = 0, total = 0;
 };
 
 int64_t n_splits_for(int64_t n_ctx) { return (n_ctx + kSplitKeys - 1) / kSplitKeys; }
@@ -92,6 +92,8 @@ WsLayout ws_layout(sdm_op op, int32_t B, int64_t N, int64_t M, int32_t H, int32_
     return w;
   }
   const int64_t rows = (op == SDM_OP_ICL_ATTENTION) ? N + M : M;
+  w.gate_w = off;  // GatedLogScale factors, one fp16 per (row, head)
+  off = align_up(off + BH * (size_t)rows * sizeof(uint16_t), kAlign);
   w.q8 = off;
   off = align_up(off + BH * (size_t)rows * kHeadDim, kAlign);
   if (op == SDM_OP_ICL_ATTENTION && !keep_cache) {
@@ -142,6 +144,7 @@ QScale make_qscale(int64_t n_len, const float* c_h, const void* gate) {
   qs.lam = logf(static_cast<float>(n_len < 1 ? 1 : n_len));
   qs.c_h = c_h;
   qs.gate = reinterpret_cast<const __half*>(gate);
+  qs.gate_w = nullptr;
   return qs;
 }
 
@@ -151,7 +154,18 @@ QScale no_qscale() {
   qs.lam = 0.0f;
   qs.c_h = nullptr;
   qs.gate = nullptr;
+  qs.gate_w = nullptr;
   return qs;
+}
+
+// With a gate, evaluate the gate factors once per (row, head) into the
+// workspace so the row kernels do not repeat the double-precision tanh per lane.
+cudaError_t prepare_gate(QScale& qs, int64_t n, uint8_t* ws_base, const WsLayout& w, cudaStream_t st) {
+  if (!qs.enabled || qs.gate == nullptr) return cudaSuccess;
+  __half* gw = reinterpret_cast<__half*>(ws_base + w.gate_w);
+  cudaError_t e = launch_gate_factors(qs.gate, n, gw, st);
+  qs.gate_w = gw;
+  return e;
 }
 
 // amax -> scales -> Q8 / K8 / V8^T.  `qs` is applied to Q (enabled: raw q in).
@@ -161,6 +175,7 @@ sdm_status run_quantize(const __half* q, const __half* k, const __half* v, int32
   const int64_t T = N + M;
   uint32_t* amax = reinterpret_cast<uint32_t*>(ws_base + w.amax);
   SDM_CUDA(cudaMemsetAsync(amax, 0, 3 * (size_t)B * H * sizeof(uint32_t), st));
+  SDM_CUDA(prepare_gate(qs, (int64_t)B * T * H, ws_base, w, st));
   RowsDesc dq{q, B, H, T}, dk{k, B, H, N}, dv{v, B, H, N};
   SDM_CUDA(launch_context_amax(dq, qs, dk, dv, N, amax, st));
   SDM_CUDA(launch_scales_from_amax(amax, B * H, scales, st));
@@ -375,7 +390,9 @@ sdm_status sdm_cached_attention(const void* q, int32_t B, int64_t M, int32_t H, 
   uint8_t* q8 = base + w.q8;
   // query scaling with the shared key length n = N, quantised with the context s_q
   RowsDesc dq{reinterpret_cast<const __half*>(q), B, H, M};
-  SDM_CUDA(launch_quantize_rows(dq, make_qscale(N, c_h, gate), M, cache->scales, q8, M, st));
+  QScale qs = make_qscale(N, c_h, gate);
+  SDM_CUDA(prepare_gate(qs, (int64_t)B * M * H, base, w, st));
+  SDM_CUDA(launch_quantize_rows(dq, qs, M, cache->scales, q8, M, st));
   AttnArgs a;
   a.B = B;
   a.H = H;
@@ -416,6 +433,7 @@ sdm_status sdm_sync_status(void* ws, void* stream, uint32_t* flags) {
 }
 
 }  // extern "C"
+
 // ---------------------------------------------------------------------------
 // Context quantisation for callers that cannot provide a workspace.
 //

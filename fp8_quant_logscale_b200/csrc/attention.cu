@@ -18,8 +18,9 @@
 //               ones in the V stage give the row sum l = sum P in O's
 //               columns 64..79, so the softmax never adds up P itself;
 //   warps 0..7  softmax, warpgroup t for tile t, one TMEM lane (= query row)
-//               per thread: row max, P = 2^(z*c2 - m2) -> e4m3 written back
-//               into TMEM over S, and O rescaled when the running max rises.
+//               per thread: all 128 logits of the tile read in one TMEM pass,
+//               row max, P = 2^(z*c2 - m2) -> e4m3 written back into TMEM over
+//               S, and O rescaled when the running max rises.
 // The two tiles ping-pong: while one warpgroup turns S into P the tensor core
 // works on the other tile.
 //
@@ -350,28 +351,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int64_t nvalid = kv_end - (kv_begin + (int64_t)it * kKvTile);
       const bool ragged = nvalid < kKvTile;
-      // pass 1: the tile's row max, 64 logits in registers at a time
+      // one read of the 128 logits: four loads in flight, one wait
+      uint32_t ra[32], rb[32], rc[32], rd[32];
+      tmem_ld_32x32b_x32(t_s, ra);
+      tmem_ld_32x32b_x32(t_s + 32, rb);
+      tmem_ld_32x32b_x32(t_s + 64, rc);
+      tmem_ld_32x32b_x32(t_s + 96, rd);
+      tmem_ld_wait();
+      if (ragged) {
+        mask_keys(ra, rb, 0, nvalid);
+        mask_keys(rc, rd, 64, nvalid);
+      }
       float mx0 = m_run, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t ra[32], rb[32];
-        tmem_ld_32x32b_x32(t_s + 64 * h, ra);
-        tmem_ld_32x32b_x32(t_s + 64 * h + 32, rb);
-        tmem_ld_wait();
-        if (ragged) mask_keys(ra, rb, 64 * h, nvalid);
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          mx0 = max3(mx0, __uint_as_float(ra[i + 0]), __uint_as_float(rb[i + 0]));
-          mx1 = max3(mx1, __uint_as_float(ra[i + 1]), __uint_as_float(rb[i + 1]));
-          mx2 = max3(mx2, __uint_as_float(ra[i + 2]), __uint_as_float(rb[i + 2]));
-          mx3 = max3(mx3, __uint_as_float(ra[i + 3]), __uint_as_float(rb[i + 3]));
+      for (int i = 0; i < 32; ++i) {
+        if (i % 2 == 0) {
+          mx0 = max3(mx0, __uint_as_float(ra[i]), __uint_as_float(rb[i]));
+          mx1 = max3(mx1, __uint_as_float(rc[i]), __uint_as_float(rd[i]));
+        } else {
+          mx2 = max3(mx2, __uint_as_float(ra[i]), __uint_as_float(rb[i]));
+          mx3 = max3(mx3, __uint_as_float(rc[i]), __uint_as_float(rd[i]));
         }
       }
       const float mt = max3(mx0, mx1, fmaxf(mx2, mx3));
       const bool up = mt > m_run;
       const float m2_new = up ? __fmul_rn(mt, c2) : m2;
+      // P = 2^(fma(z, c2, -m2)) in (0, 1] -> e4m3, four codes per 32-bit TMEM
+      // column, written over S columns whose logits are already in registers
+      const float nm2 = -m2_new;
+      {
+        uint32_t pw[16];
+        p_words<0>(ra, rb, pw, c2, nm2);
+        tmem_st_32x32b_x16(t_s, pw);
+      }
+      {
+        uint32_t pw[16];
+        p_words<0>(rc, rd, pw, c2, nm2);
+        tmem_st_32x32b_x16(t_s + 16, pw);
+      }
       if (it > 0 && __any_sync(0xffffffffu, up)) {
-        // O and its row sum were accumulated against the old max: rescale.
+        // O and its row sum were accumulated against the old max: rescale (after
+        // the P stores, so the logits' registers are free again).
         const float alpha = up ? ex2_approx(__fsub_rn(m2, m2_new)) : 1.0f;
         uint32_t o[32];
 #pragma unroll
@@ -389,20 +409,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       m_run = mt;
       m2 = m2_new;
-      // pass 2: P = 2^(fma(z, c2, -m2)) in (0, 1] -> e4m3, four codes per
-      // 32-bit TMEM column, written over S columns that are already consumed
-      const float nm2 = -m2;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t ra[32], rb[32];
-        tmem_ld_32x32b_x32(t_s + 64 * h, ra);
-        tmem_ld_32x32b_x32(t_s + 64 * h + 32, rb);
-        tmem_ld_wait();
-        if (ragged) mask_keys(ra, rb, 64 * h, nvalid);
-        uint32_t pw[16];
-        p_words<0>(ra, rb, pw, c2, nm2);
-        tmem_st_32x32b_x16(t_s + 16 * h, pw);
-      }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();

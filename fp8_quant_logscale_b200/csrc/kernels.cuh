@@ -19,6 +19,7 @@ struct QScale {
   float lam;           // fp32 ln(max(n,1)), evaluated on the host from the integer length
   const float* c_h;    // [H] per-head coefficients (device)
   const __half* gate;  // [B][rows][H] or nullptr (LogScale)
+  const __half* gate_w;  // [B][rows][H] precomputed fp16(1 + fp16(tanh g)), or nullptr: evaluate in place
 };
 
 // Tensor-wide problem description for the elementwise kernels.
@@ -30,6 +31,9 @@ struct RowsDesc {
 
 cudaError_t launch_qscale(const __half* q, __half* out, int32_t B, int64_t rows, int32_t H, QScale qs,
                           cudaStream_t st);
+
+// w[i] = fp16(1 + fp16(tanh(gate[i]))) for i < n: the GatedLogScale factor, once per (row, head).
+cudaError_t launch_gate_factors(const __half* gate, int64_t n, __half* w, cudaStream_t st);
 
 // amax words: [3][B][H] uint32 (float bits, values >= 0).  Must be zeroed first.
 cudaError_t launch_context_amax(RowsDesc q, QScale qs, RowsDesc k, RowsDesc v, int64_t n_ctx, uint32_t* amax,

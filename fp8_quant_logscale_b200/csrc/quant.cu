@@ -23,11 +23,15 @@ __device__ __forceinline__ float head_scale(const QScale& qs, int h) {
   return __half2float(__float2half_rn(__fmul_rn(__ldg(qs.c_h + h), qs.lam)));
 }
 
+// w = fp16(1 + fp16(tanh g)); tanh evaluated in double and rounded once to fp16.
+__device__ __forceinline__ __half gate_factor_of(__half g) {
+  const __half u = __double2half(tanh(static_cast<double>(__half2float(g))));
+  return __float2half_rn(__fadd_rn(1.0f, __half2float(u)));
+}
+
 __device__ __forceinline__ float gate_factor(const QScale& qs, int64_t br, int H, int h) {
-  // w = fp16(1 + fp16(tanh g)); tanh evaluated in double and rounded once to fp16.
-  const float g = __half2float(qs.gate[br * H + h]);
-  const __half u = __double2half(tanh(static_cast<double>(g)));
-  return __half2float(__float2half_rn(__fadd_rn(1.0f, __half2float(u))));
+  if (qs.gate_w != nullptr) return __half2float(qs.gate_w[br * H + h]);
+  return __half2float(gate_factor_of(qs.gate[br * H + h]));
 }
 
 // One fp16 element through the eager chain: q1 = fp16(q*s), gated: fp16(q1*w).
@@ -35,6 +39,30 @@ __device__ __forceinline__ float qscale1(float q, float s, bool gated, float w) 
   float q1 = __half2float(__float2half_rn(__fmul_rn(q, s)));
   if (gated) q1 = __half2float(__float2half_rn(__fmul_rn(q1, w)));
   return q1;
+}
+
+// x / s correctly rounded, for a divisor s > 0 that stays fixed over many x:
+// with y = RN(1/s) and q = RN(x*y), the remainder r = x - q*s is exact in one
+// fma and RN(q + r*y) equals RN(x/s) (Markstein's correction step, IEEE
+// binary32, valid while nothing under- or overflows: here |x/s| <= 448 and
+// s >= 2^-33).  The one case it gets wrong is the sign of a zero (x = -0 gives
+// +0 + -0 = +0), so the result takes x's sign, which is the sign of x/s for
+// every x because s > 0.  Three FMA-pipe operations per pair of elements plus a
+// sign copy each, instead of a division each.
+struct Divider {
+  float y, neg_s;
+};
+__device__ __forceinline__ Divider make_divider(float s) { return {__frcp_rn(s), -s}; }
+__device__ __forceinline__ void divide8(float (&f)[8], const Divider& d) {
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    float q0, q1, r0, r1, d0, d1;
+    mul2(q0, q1, f[i], f[i + 1], d.y, d.y);
+    fma2(r0, r1, q0, q1, d.neg_s, d.neg_s, f[i], f[i + 1]);
+    fma2(d0, d1, r0, r1, d.y, d.y, q0, q1);
+    f[i] = copysignf(d0, f[i]);
+    f[i + 1] = copysignf(d1, f[i + 1]);
+  }
 }
 
 __device__ __forceinline__ void unpack8(const uint4& raw, float (&f)[8]) {
@@ -96,6 +124,12 @@ __global__ void __launch_bounds__(256) qscale_kernel(const __half* __restrict__ 
       __stcs(reinterpret_cast<uint4*>(out) + i, res);
     }
   }
+}
+
+__global__ void __launch_bounds__(256) gate_factor_kernel(const __half* __restrict__ gate, int64_t n,
+                                                          __half* __restrict__ w) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    w[i] = gate_factor_of(gate[i]);
 }
 
 // ------------------------------------------------------------ context amax
@@ -174,7 +208,7 @@ __global__ void quantize_rows_kernel(RowsDesc X, QScale qs, int64_t n_rows, cons
   const int64_t r0 = (blockIdx.x % chunks) * rows_per_cta;
   const int64_t r1 = min(n_rows, r0 + rows_per_cta);
   const float s = do_q ? head_scale(qs, h) : 1.0f;
-  const float sx = __ldg(scale + b * H + h);
+  const Divider dv = make_divider(__ldg(scale + b * H + h));
   uint8_t* dbase = dst + ((int64_t)b * H + h) * dst_rows * kHeadDim + j * 8;
   for (int64_t r = r0 + t / vecs_per_row; r < r1; r += kUnroll * row_step) {
     uint4 raw[kUnroll];
@@ -190,8 +224,11 @@ __global__ void quantize_rows_kernel(RowsDesc X, QScale qs, int64_t n_rows, cons
       const float w = gated ? gate_factor(qs, (int64_t)b * X.rows + rr, H, h) : 1.0f;
       float f[8];
       unpack8(raw[u], f);
+      if (do_q) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) f[e] = __fdiv_rn(do_q ? qscale1(f[e], s, gated, w) : f[e], sx);
+        for (int e = 0; e < 8; ++e) f[e] = qscale1(f[e], s, gated, w);
+      }
+      divide8(f, dv);
       uint2 codes;
       codes.x = e4m3x2(f[0], f[1]) | (e4m3x2(f[2], f[3]) << 16);
       codes.y = e4m3x2(f[4], f[5]) | (e4m3x2(f[6], f[7]) << 16);
@@ -210,7 +247,7 @@ __global__ void __launch_bounds__(256) quantize_vt_kernel(RowsDesc V, int64_t n_
   const int64_t bh = blockIdx.y;
   const int b = static_cast<int>(bh / H), h = static_cast<int>(bh % H);
   const int64_t r0 = (int64_t)blockIdx.x * kKvTile;
-  const float sx = __ldg(scale + bh);
+  const Divider dv = make_divider(__ldg(scale + bh));
   const int t = threadIdx.x;
   const int j = t & 7;  // elements 8j..8j+7
   uint8_t* tb = reinterpret_cast<uint8_t*>(&tile[0][0]);
@@ -229,8 +266,7 @@ __global__ void __launch_bounds__(256) quantize_vt_kernel(RowsDesc V, int64_t n_
     if (r < n_ctx) {
       float f[8];
       unpack8(raws[i], f);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) f[e] = __fdiv_rn(f[e], sx);
+      divide8(f, dv);
       lo = e4m3x2(f[0], f[1]) | (e4m3x2(f[2], f[3]) << 16);
       hi = e4m3x2(f[4], f[5]) | (e4m3x2(f[6], f[7]) << 16);
     }
@@ -263,6 +299,14 @@ cudaError_t launch_qscale(const __half* q, __half* out, int32_t B, int64_t rows,
   const int64_t want = (n_vec + 256 * kUnroll - 1) / (256 * kUnroll);
   const int grid = static_cast<int>(want < (int64_t)num_sms() * 8 ? want : (int64_t)num_sms() * 8);
   qscale_kernel<<<grid, 256, 0, st>>>(q, out, n_vec, H, qs);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gate_factors(const __half* gate, int64_t n, __half* w, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const int64_t want = (n + 255) / 256;
+  const int grid = static_cast<int>(want < (int64_t)num_sms() * 8 ? want : (int64_t)num_sms() * 8);
+  gate_factor_kernel<<<grid, 256, 0, st>>>(gate, n, w);
   return cudaGetLastError();
 }
 

@@ -37,3 +37,25 @@ def test_quantize_with_outliers(cuda_lib, orc):
     inp = make_inputs(WORKLOADS["icl_n128k_m1k_h8_gated"], n_ctx=8192, n_query=256)
     qs = orc.qscale(inp["q"], 8192, inp["c_h"], inp["gate"])
     _check(cuda_lib, orc, qs, inp["k"], inp["v"], 8192)
+
+
+def test_quotients_of_every_fp16_value(cuda_lib, orc):
+    """Every finite fp16 value (up to each head's amax) divided by 256 different
+    context scales, through the Q/K row and the transposed V quantisers: the
+    e4m3 codes must equal those of an IEEE fp32 division in the oracle."""
+    B, H = 4, 64
+    vals = np.arange(0, 0x7C00, dtype=np.uint16).view(np.float16)      # +0 .. 65504
+    vals = np.concatenate([vals, -vals]).astype(np.float16)              # -0 too: its code is 0x80
+    rows = (vals.size + 63) // 64
+    flat = np.zeros(rows * 64, np.float16)
+    flat[:vals.size] = vals
+    rng = np.random.default_rng(42)
+    # per-(b, h) amax: random fp16 magnitudes from subnormal to max
+    amax = np.abs(rng.choice(vals[vals != 0], B * H)).astype(np.float16)
+    x = np.empty((B, rows, H, 64), np.float16)
+    base = flat.reshape(rows, 64).astype(np.float32)
+    for i in range(B * H):
+        b, h = divmod(i, H)
+        a = np.float32(amax[i])
+        x[b, :, h, :] = np.clip(base, -a, a).astype(np.float16)
+    _check(cuda_lib, orc, x, x.copy(), x.copy(), rows)
