@@ -26,7 +26,7 @@ HEAD_DIM = 64
 # Every symbol the header declares (checked by the ABI tests).
 EXPORTS = ("sdm_status_string", "sdm_version", "sdm_cache_layout", "sdm_workspace_size", "sdm_qscale_fused",
            "sdm_fp8_quantize_context", "sdm_fp8_quantize_context_noalloc", "sdm_fp8_attention", "sdm_icl_attention",
-           "sdm_cached_attention", "sdm_sync_status")
+           "sdm_cached_attention", "sdm_sync_status", "sdm_selftest_wait_timeout")
 NOALLOC_MAX_BATCH_HEADS = 4096
 
 
@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
         L.sdm_cached_attention.restype = ctypes.c_int
         L.sdm_cached_attention.argtypes = [_P, _I32, _I64, _I32, _I32, ctypes.POINTER(CacheStruct), _P, _P, _P,
                                            _P, _SZ, _P]
+        L.sdm_selftest_wait_timeout.restype = ctypes.c_int
+        L.sdm_selftest_wait_timeout.argtypes = [_P, _I64, _P]
         L.sdm_sync_status.restype = ctypes.c_int
         L.sdm_sync_status.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_uint32)]
         _lib = L
@@ -131,6 +133,13 @@ def sync_status(ws: torch.Tensor) -> tuple[int, int]:
     flags = ctypes.c_uint32(0)
     st = lib().sdm_sync_status(_ptr(ws), _stream(ws.device), ctypes.byref(flags))
     return int(st), int(flags.value)
+
+
+def selftest_wait_timeout(ws: torch.Tensor, limit_cycles: int = 1_000_000) -> None:
+    """Enqueue the bounded-wait self-test on `ws` (see sdm_selftest_wait_timeout)."""
+    with torch.cuda.device(ws.device):
+        _check(lib().sdm_selftest_wait_timeout(_ptr(ws), int(limit_cycles), _stream(ws.device)),
+               "sdm_selftest_wait_timeout")
 
 
 class FP8Cache:

@@ -412,6 +412,16 @@ sdm_status sdm_cached_attention(const void* q, int32_t B, int64_t M, int32_t H, 
   return SDM_OK;
 }
 
+sdm_status sdm_selftest_wait_timeout(void* ws, int64_t limit_cycles, void* stream) {
+  if (ws == nullptr || !aligned(ws, 256)) return SDM_ERR_INVALID_ARG;
+  if (limit_cycles < 1000 || limit_cycles > ((int64_t)1 << 31)) return SDM_ERR_INVALID_ARG;
+  const int dev = current_device();
+  if (dev < 0) return SDM_ERR_CUDA;
+  if (!on_device(ws, dev)) return SDM_ERR_DEVICE_MISMATCH;
+  SDM_CUDA(launch_wait_selftest(reinterpret_cast<uint32_t*>(ws), limit_cycles, as_stream(stream)));
+  return SDM_OK;
+}
+
 sdm_status sdm_sync_status(void* ws, void* stream, uint32_t* flags) {
   if (ws == nullptr) return SDM_ERR_INVALID_ARG;
   cudaStream_t st = as_stream(stream);

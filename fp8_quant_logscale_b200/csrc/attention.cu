@@ -24,7 +24,10 @@
 // The two tiles ping-pong: while one warpgroup turns S into P the tensor core
 // works on the other tile.
 //
-// TMEM (512 columns): S0 [0,128)  S1 [128,256)  O0 [256,336)  O1 [336,416).
+// TMEM (512 columns): S0 [0,128)  S1 [128,256)  O0 [256,336)  O1 [336,416)
+//                     P0 [416,448)  P1 [448,480).
+// P has its own columns, so the next S = Q K^T is issued as soon as the
+// softmax has read S into registers and overlaps the softmax arithmetic.
 #include <math.h>
 
 #include "exp2_poly.cuh"
@@ -50,6 +53,7 @@ constexpr int kVLoadBytes = kHeadDim * kKvTile;   // 8 KB loaded by TMA
 constexpr uint32_t kTmemCols = 512;
 __device__ __forceinline__ uint32_t s_col(int t) { return 128u * t; }
 __device__ __forceinline__ uint32_t o_col(int t) { return 256u + 80u * t; }
+__device__ __forceinline__ uint32_t p_col(int t) { return 416u + 32u * t; }
 
 constexpr long long kWaitLimit = 1LL << 31;   // ~1 s of SM clock: no legitimate wait comes close
 constexpr long long kDrainLimit = 1LL << 24;  // teardown waits for copies in flight
@@ -62,9 +66,10 @@ struct __align__(1024) Smem {
   uint64_t k_full[kStages];
   uint64_t v_full[kStages];
   uint64_t kv_empty[kStages];
-  uint64_t s_full[kTiles];
-  uint64_t p_full[kTiles];
-  uint64_t o_full[kTiles];
+  uint64_t s_full[kTiles];   // S_t = Q_t K^T landed in TMEM
+  uint64_t s_free[kTiles];   // the softmax holds S_t in registers: the next QK may overwrite it
+  uint64_t p_full[kTiles];   // P_t stored in TMEM (and O_t rescaled)
+  uint64_t o_ready[kTiles];  // O_t += P_t V done: P_t may be overwritten, O_t read
   uint64_t drain;
   uint32_t tmem_base;
   uint32_t abort_flag;
@@ -202,8 +207,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < kTiles; ++t) {
       mbar_init(&s.s_full[t], 1);
-      mbar_init(&s.p_full[t], 4);  // one arrival per softmax warp
-      mbar_init(&s.o_full[t], 1);
+      mbar_init(&s.s_free[t], 4);  // one arrival per softmax warp
+      mbar_init(&s.p_full[t], 4);
+      mbar_init(&s.o_ready[t], 1);
     }
     mbar_init(&s.drain, 1);
     s.abort_flag = 0u;
@@ -271,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t b0 = smem_u32(s.v[st]);
 #pragma unroll
         for (int ks = 0; ks < kKvTile / 32; ++ks)
-          mma_e4m3_ts(tmem + o_col(t), tmem + s_col(t) + 8 * ks, smem_desc_kmajor(b0 + 32 * ks, 1024, kSwizzle128B),
+          mma_e4m3_ts(tmem + o_col(t), tmem + p_col(t) + 8 * ks, smem_desc_kmajor(b0 + 32 * ks, 1024, kSwizzle128B),
                       idesc_o, (acc || ks > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(&s.q_full, 0, abort_flag, kWaitLimit);
@@ -287,17 +293,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&s.s_full[t]);
         }
       }
+      // Per tile t and key tile it: as soon as the softmax holds S_t(it) in
+      // registers, issue S_t(it+1) = Q_t K(it+1)^T, so it overlaps the softmax
+      // arithmetic; when P_t(it) is stored, issue O_t += P_t(it) V(it).
       for (int it = 0; ok && it < n_tiles; ++it) {
         const int st = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
         const int nst = (it + 1) % kStages;
         const uint32_t nph = ((it + 1) / kStages) & 1;
+        const bool more = it + 1 < n_tiles;
+        if (more && !mbar_wait(&s.k_full[nst], nph, abort_flag, kWaitLimit)) {
+          raise_abort(s, p.err, kErrTimeoutKV);
+          ok = false;
+          break;
+        }
         if (!mbar_wait(&s.v_full[st], ph, abort_flag, kWaitLimit)) {
           raise_abort(s, p.err, kErrTimeoutKV);
           ok = false;
           break;
         }
         for (int t = 0; t < kTiles; ++t) {
+          if (more) {
+            if (!mbar_wait(&s.s_free[t], it & 1, abort_flag, kWaitLimit)) {
+              raise_abort(s, p.err, kErrTimeoutS);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_qk(t, nst);
+            mma_commit(&s.s_full[t]);
+          }
           if (!mbar_wait(&s.p_full[t], it & 1, abort_flag, kWaitLimit)) {
             raise_abort(s, p.err, kErrTimeoutP);
             ok = false;
@@ -305,22 +330,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           issue_pv(t, st, it > 0);
-          if (t == kTiles - 1) mma_commit(&s.kv_empty[st]);
-          if (it + 1 < n_tiles) {
-            if (t == 0) {
-              if (!mbar_wait(&s.k_full[nst], nph, abort_flag, kWaitLimit)) {
-                raise_abort(s, p.err, kErrTimeoutKV);
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-            }
-            issue_qk(t, nst);
-            mma_commit(&s.s_full[t]);
-          } else {
-            mma_commit(&s.o_full[t]);
-          }
+          mma_commit(&s.o_ready[t]);
         }
+        if (ok) mma_commit(&s.kv_empty[st]);  // K(it) and V(it) consumed by both tiles
       }
       // teardown: every MMA issued must complete before TMEM is released
       mma_commit(&s.drain);
@@ -332,6 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wq = warp & 3;   // TMEM lane quadrant
     const uint32_t lane_base = static_cast<uint32_t>(32 * wq) << 16;
     const uint32_t t_s = tmem + lane_base + s_col(t);
+    const uint32_t t_p = tmem + lane_base + p_col(t);
     const uint32_t t_o = tmem + lane_base + o_col(t);
     const float s_q = __ldg(p.scales + bh);
     const float s_k = __ldg(p.scales + p.BH + bh);
@@ -358,6 +371,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld_32x32b_x32(t_s + 64, rc);
       tmem_ld_32x32b_x32(t_s + 96, rd);
       tmem_ld_wait();
+      // S_t is in registers: the tensor core may compute the next S_t now
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.s_free[t]);
       if (ragged) {
         mask_keys(ra, rb, 0, nvalid);
         mask_keys(rc, rd, 64, nvalid);
@@ -376,18 +393,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float mt = max3(mx0, mx1, fmaxf(mx2, mx3));
       const bool up = mt > m_run;
       const float m2_new = up ? __fmul_rn(mt, c2) : m2;
-      // P = 2^(fma(z, c2, -m2)) in (0, 1] -> e4m3, four codes per 32-bit TMEM
-      // column, written over S columns whose logits are already in registers
+      // the previous P_t V must be done before P_t is overwritten and O_t rescaled
+      if (it > 0) {
+        ok = mbar_wait(&s.o_ready[t], (it - 1) & 1, abort_flag, kWaitLimit);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) {
+          if (lane == 0) raise_abort(s, p.err, kErrTimeoutO);
+          break;
+        }
+        tc_fence_after();
+      }
+      // P = 2^(fma(z, c2, -m2)) in (0, 1] -> e4m3, four codes per 32-bit TMEM column
       const float nm2 = -m2_new;
       {
         uint32_t pw[16];
         p_words<0>(ra, rb, pw, c2, nm2);
-        tmem_st_32x32b_x16(t_s, pw);
+        tmem_st_32x32b_x16(t_p, pw);
       }
       {
         uint32_t pw[16];
         p_words<0>(rc, rd, pw, c2, nm2);
-        tmem_st_32x32b_x16(t_s + 16, pw);
+        tmem_st_32x32b_x16(t_p + 16, pw);
       }
       if (it > 0 && __any_sync(0xffffffffu, up)) {
         // O and its row sum were accumulated against the old max: rescale (after
@@ -416,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ---- epilogue
     if (ok && n_tiles > 0) {
-      ok = mbar_wait(&s.o_full[t], 0, abort_flag, kWaitLimit);
+      ok = mbar_wait(&s.o_ready[t], (n_tiles - 1) & 1, abort_flag, kWaitLimit);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok && lane == 0) raise_abort(s, p.err, kErrTimeoutO);
     }
@@ -503,6 +529,23 @@ __global__ void __launch_bounds__(256) splitkv_reduce_kernel(const float* __rest
   reinterpret_cast<__half2*>(out + ((b * T + row) * H + h) * kHeadDim)[lane] = hv;
 }
 
+// ------------------------------------------------------------ wait self-test
+// The failure path of every bounded wait above, exercised on purpose: the
+// barrier below never completes, so the wait gives up after `limit` cycles and
+// the kernel reports it through the error word and returns.
+__global__ void wait_selftest_kernel(uint32_t* err, long long limit) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0u;
+    fence_mbar_init();
+  }
+  __syncwarp();
+  const bool ok = mbar_wait(&bar, 0, &abort_flag, limit);
+  if (!ok && threadIdx.x == 0) atomicOr(err, kErrTimeoutSelfTest);
+}
+
 // ------------------------------------------------------------ host helpers
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -583,4 +626,11 @@ cudaError_t launch_splitkv_reduce(const AttnArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+}  // namespace sdm
+
+namespace sdm {
+cudaError_t launch_wait_selftest(uint32_t* err, long long limit, cudaStream_t st) {
+  wait_selftest_kernel<<<1, 32, 0, st>>>(err, limit);
+  return cudaGetLastError();
+}
 }  // namespace sdm

@@ -81,5 +81,10 @@ constexpr uint32_t kErrTimeoutP = 1u << 3;
 constexpr uint32_t kErrTimeoutO = 1u << 4;
 constexpr uint32_t kErrTimeoutEmpty = 1u << 5;
 constexpr uint32_t kErrTimeoutDrain = 1u << 6;
+constexpr uint32_t kErrTimeoutSelfTest = 1u << 7;
+
+// One warp waits, with the kernels' bounded wait, on an mbarrier that nothing
+// arrives at; when `limit` cycles pass it ORs kErrTimeoutSelfTest into *err.
+cudaError_t launch_wait_selftest(uint32_t* err, long long limit, cudaStream_t st);
 
 }  // namespace sdm

@@ -233,6 +233,16 @@ sdm_status sdm_fp8_quantize_context_noalloc(const void* q_scaled, const void* k,
  */
 sdm_status sdm_sync_status(void* ws, void* stream, uint32_t* flags);
 
+/*
+ * Self-test of the failure path shared by every in-kernel wait: launches one
+ * warp that waits, with the same bounded mbarrier wait the attention kernel
+ * uses, on a barrier that nothing ever arrives at.  After `limit_cycles` SM
+ * clock cycles (1000 .. 2^31) the wait gives up, the kernel sets bit 7 of the
+ * error word at the head of `ws` and returns; sdm_sync_status() then reports
+ * SDM_ERR_TIMEOUT and the CUDA context stays usable.  Nothing faults or hangs.
+ */
+sdm_status sdm_selftest_wait_timeout(void* ws, int64_t limit_cycles, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -53,3 +53,20 @@ def test_small_workspace(cuda_lib):
     assert e.value.status == 3
     st, flags = cuda_lib.sync_status(ws)
     assert st == 0 and flags == 0
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(cuda_lib):
+    """A wait that can never complete gives up after its cycle limit: the error
+    word says so, sdm_sync_status returns SDM_ERR_TIMEOUT, the word is cleared,
+    and the next call on the same context works."""
+    ws = cuda_lib.new_workspace(256, "cuda")
+    binding.selftest_wait_timeout(ws, limit_cycles=2_000_000)
+    st, flags = cuda_lib.sync_status(ws)
+    assert st == 6 and flags == 1 << 7
+    assert cuda_lib.sync_status(ws) == (0, 0)
+    q, k, c = _small(cuda_lib)
+    out = cuda_lib.icl_attention(q, k, k, 256, c)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
+    L = binding.lib()
+    assert L.sdm_selftest_wait_timeout(ctypes.c_void_p(ws.data_ptr()), 10, None) == 1   # limit too small
