@@ -37,6 +37,23 @@ FP8_NOMINAL_TFLOPS = 4500.0
 BF16_NOMINAL_TFLOPS = 2250.0
 
 
+# DRAM bytes (read + write) of one fit launch of the attention kernel on the
+# 512K workload, from a one-pass ncu capture (profiles/icl_attention_kernel_n512k_dram.md).
+# Valid only for the kernel source it was taken on: any change to these files
+# makes the bench report null until a new capture is recorded here.
+ATTN_TRAFFIC_SOURCES = ("attention.cu", "ptx.cuh", "exp2_poly.cuh", "kernels.cuh")
+ATTN_TRAFFIC = {"source_sha256": None, "bytes": None}
+
+
+def attention_source_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in ATTN_TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, "fp8_quant_logscale_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def attn_flops(rows: int, n_ctx: int, heads: int, d: int = 64) -> float:
     """Algorithmic FLOPs of one attention: S = QK^T and O = PV, 2*d each per (row, key, head)."""
     return 4.0 * d * heads * rows * n_ctx
@@ -274,8 +291,18 @@ def run_ours(args):
     else:
         fp8_peak = 1400.0 * 2
         peak_src = "of fallback (1.4 PF bf16 sustained x 2)"
+    traffic = args.traffic
+    if traffic is None and args.workload == DEFAULT_WORKLOAD and ATTN_TRAFFIC["bytes"] is not None \
+            and attention_source_sha256() == ATTN_TRAFFIC["source_sha256"]:
+        traffic = ATTN_TRAFFIC["bytes"]
     kmean = statistics.mean(kern_ms)
     achieved = attn_flops(T, N, H) / (kmean * 1e-3) / 1e12
+    clocks = clk.summary()
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0
+    # The softmax's own ceiling: one 2^x per (row, key, head) on the MUFU pipe
+    # (16 per clock per SM) against 4*64 = 256 tensor FLOP per logit.
+    mufu_tflops = 16 * 4 * 64 * sms * mhz * 1e6 / 1e12
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -288,10 +315,12 @@ def run_ours(args):
         "attention_kernel_ms": kmean,
         "pct_fp8_peak": 100.0 * achieved / fp8_peak, "pct_fp8_nominal": 100.0 * achieved / FP8_NOMINAL_TFLOPS,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
-                     "frac": achieved / fp8_peak, "traffic": args.traffic, "peak_source": peak_src,
+                     "frac": achieved / fp8_peak, "traffic": traffic, "peak_source": peak_src,
                      "kernel": "icl_attention_kernel (FP8 attention of all rows)"},
+        "softmax_bound": {"kind": "MUFU ex2, 16/clk/SM, one per logit", "peak": mufu_tflops, "unit": "TFLOP/s",
+                          "frac": achieved / mufu_tflops, "sm_mhz": mhz, "sms": sms},
         "gpu_launches": args.steps * 9,
-        "clocks": clk.summary(),
+        "clocks": clocks,
     }
     if e2e:
         line["e2e"] = e2e
@@ -304,6 +333,77 @@ def run_ours(args):
     import torch.distributed as dist
     if dist.is_initialized():
         dist.destroy_process_group()
+
+
+# ------------------------------------------------------------- per kernel
+def run_per_kernel(args):
+    """Each step of the path alone, through its C-ABI entry point, timed with CUDA
+    events (median of K after W warm-ups) on the chosen workload; one JSON line per step."""
+    import torch
+
+    import fp8_quant_logscale_b200 as sdm
+    from fp8_quant_logscale_b200 import binding
+    from fp8_quant_logscale_b200.workloads import WORKLOADS, make_inputs
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w)
+    B, N, M, H = inp["B"], inp["N"], inp["M"], inp["H"]
+    T = N + M
+    q = torch.from_numpy(inp["q"]).to(device)
+    k = torch.from_numpy(inp["k"]).to(device)
+    v = torch.from_numpy(inp["v"]).to(device)
+    c_h = torch.from_numpy(inp["c_h"]).to(device)
+    gate = None if inp["gate"] is None else torch.from_numpy(inp["gate"]).to(device)
+    qs = torch.empty_like(q)
+    out = torch.empty_like(q)
+    cache = sdm.FP8Cache(B, N, H, device)
+    q8 = torch.empty((B, H, T, 64), dtype=torch.uint8, device=device)
+    ws_q = sdm.new_workspace(sdm.workspace_size(binding.OP_QUANTIZE_CONTEXT, B, N, M, H), device)
+    ws_a = sdm.new_workspace(256, device)
+    Mq = 1024
+    queries = q[:, :Mq].contiguous()
+    pred = torch.empty_like(queries)
+    ws_c = sdm.new_workspace(sdm.workspace_size(binding.OP_CACHED_ATTENTION, B, N, Mq, H), device)
+    stream = torch.cuda.current_stream(device)
+    peaks = measured_peaks() or {"hbm_gbs": 6650.0, "bf16_tflops_sustained": 1400.0}
+    hbm = peaks["hbm_gbs"]
+    fp8 = peaks["bf16_tflops_sustained"] * FP8_NOMINAL_TFLOPS / BF16_NOMINAL_TFLOPS
+    el = lambda rows: B * rows * H * 64
+    steps = [
+        # name, call, algorithmic bytes, flops
+        ("a1 qscale (sdm_qscale_fused)", lambda: sdm.qscale_fused(q, c_h, N, gate, out=qs),
+         4 * el(T) + (2 * B * T * H if gate is not None else 0), 0.0),
+        ("a2 context quantisation (sdm_fp8_quantize_context)",
+         lambda: sdm.fp8_quantize_context(qs, k, v, N, cache=cache, ws=ws_q),
+         # amax pass reads the context rows of Q', K, V (2 B); the quantise pass reads
+         # all of them again and writes e4m3 (3 B): both passes are inherent
+         2 * 3 * el(N) + 3 * (el(T) + 2 * el(N)), 0.0),
+        ("a3 FP8 attention (sdm_fp8_attention)", lambda: sdm.fp8_attention(q8, cache, out=out, ws=ws_a),
+         el(T) + 2 * el(N) + 2 * el(T), attn_flops(T, N, H)),
+        ("a4 cached prediction, 1024 queries (sdm_cached_attention)",
+         lambda: sdm.cached_attention(queries, cache, c_h, gate=None, out=pred, ws=ws_c),
+         2 * el(Mq) + 2 * el(N) + 2 * el(Mq), attn_flops(Mq, N, H)),
+    ]
+    # a filled cache and Q8 for the attention steps
+    q8.copy_(sdm.fp8_quantize_context(sdm.qscale_fused(q, c_h, N, gate), k, v, N, cache=cache)[0])
+    for name, fn, nbytes, flops in steps:
+        times = []
+        for i in range(args.warmup + args.steps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize(device)
+            if i >= args.warmup:
+                times.append(a.elapsed_time(b))
+        ms = statistics.median(times)
+        line = {"step": name, "workload": w.name, "ms": ms, "bytes": nbytes,
+                "gbs": nbytes / (ms * 1e-3) / 1e9, "frac_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm}
+        if flops:
+            line.update({"tflops": flops / (ms * 1e-3) / 1e12, "frac_fp8": flops / (ms * 1e-3) / 1e12 / fp8})
+        print(json.dumps(line), flush=True)
 
 
 # ------------------------------------------------------------- reference
@@ -356,11 +456,15 @@ def main(argv=None):
     ap.add_argument("--cpu-rows", type=int, default=64, help="rows of the oracle's timed sample")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--per-kernel", action="store_true",
+                    help="time each step of the path alone (one JSON line per step) instead of the benchmark step")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per attention launch from an ncu capture of the current kernel")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         run_reference(args)
+    elif args.per_kernel:
+        run_per_kernel(args)
     else:
         run_ours(args)
 

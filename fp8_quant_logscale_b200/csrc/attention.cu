@@ -38,11 +38,18 @@ namespace sdm {
 namespace {
 
 constexpr int kStages = 4;
-constexpr int kTiles = 2;                 // query tiles per CTA
-constexpr int kSoftmaxWarps = 4 * kTiles;
-constexpr int kProducerWarp = kSoftmaxWarps;
-constexpr int kMmaWarp = kSoftmaxWarps + 1;
-constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+// Query tiles per CTA (template parameter kTiles): 2 for the general case (the
+// two tiles interleave on the tensor core), 1 when a launch has at most 128
+// rows (small prediction batches), which also lets two CTAs share an SM.
+template <int kTiles>
+struct Cfg {
+  static constexpr int kSoftmaxWarps = 4 * kTiles;
+  static constexpr int kProducerWarp = kSoftmaxWarps;
+  static constexpr int kMmaWarp = kSoftmaxWarps + 1;
+  static constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+  static constexpr uint32_t kTmemCols = kTiles == 2 ? 512 : 256;
+  static constexpr int kMinBlocks = kTiles == 2 ? 1 : 2;
+};
 
 constexpr int kQBytes = kQTile * kHeadDim;        // 8 KB, 64-byte rows
 constexpr int kKBytes = kKvTile * kHeadDim;       // 8 KB, 64-byte rows
@@ -50,14 +57,18 @@ constexpr int kVRows = kHeadDim + 16;             // V^T rows + 16 rows of ones
 constexpr int kVBytes = kVRows * kKvTile;         // 10 KB, 128-byte rows
 constexpr int kVLoadBytes = kHeadDim * kKvTile;   // 8 KB loaded by TMA
 
-constexpr uint32_t kTmemCols = 512;
+// TMEM columns: S_t at 128t, O_t after all S, P_t after all O.
+template <int kTiles>
 __device__ __forceinline__ uint32_t s_col(int t) { return 128u * t; }
-__device__ __forceinline__ uint32_t o_col(int t) { return 256u + 80u * t; }
-__device__ __forceinline__ uint32_t p_col(int t) { return 416u + 32u * t; }
+template <int kTiles>
+__device__ __forceinline__ uint32_t o_col(int t) { return 128u * kTiles + 80u * t; }
+template <int kTiles>
+__device__ __forceinline__ uint32_t p_col(int t) { return 208u * kTiles + 32u * t; }
 
 constexpr long long kWaitLimit = 1LL << 31;   // ~1 s of SM clock: no legitimate wait comes close
 constexpr long long kDrainLimit = 1LL << 24;  // teardown waits for copies in flight
 
+template <int kTiles>
 struct __align__(1024) Smem {
   uint8_t q[kTiles][kQBytes];
   uint8_t k[kStages][kKBytes];
@@ -87,7 +98,8 @@ struct KParams {
   uint32_t* err;
 };
 
-__device__ __forceinline__ void raise_abort(Smem& s, uint32_t* err, uint32_t code) {
+template <class S>
+__device__ __forceinline__ void raise_abort(S& s, uint32_t* err, uint32_t code) {
   atomicOr(err, code);
   *reinterpret_cast<volatile uint32_t*>(&s.abort_flag) = 1u;
 }
@@ -165,22 +177,34 @@ __device__ __forceinline__ uint32_t p_word(const uint32_t* z, float c2, float nm
   return e4m3x2(p0, p1) | (e4m3x2(p2, p3) << 16);
 }
 
-// Words W..7 of two 32-key chunks (compile-time word index selects the 2^x path).
+// Words W..7 of the four 32-key chunks of a tile (the compile-time word index
+// selects the 2^x path); chunk c's word w lands in TMEM column 8c + w.
 template <int W>
-__device__ __forceinline__ void p_words(const uint32_t (&ra)[32], const uint32_t (&rb)[32], uint32_t (&pw)[16],
-                                        float c2, float nm2) {
+__device__ __forceinline__ void p_words32(const uint32_t (&ra)[32], const uint32_t (&rb)[32], const uint32_t (&rc)[32],
+                                          const uint32_t (&rd)[32], uint32_t (&pw)[32], float c2, float nm2) {
   if constexpr (W < 8) {
     pw[W] = p_word<poly_word(W)>(ra + 4 * W, c2, nm2);
     pw[8 + W] = p_word<poly_word(W)>(rb + 4 * W, c2, nm2);
-    p_words<W + 1>(ra, rb, pw, c2, nm2);
+    pw[16 + W] = p_word<poly_word(W)>(rc + 4 * W, c2, nm2);
+    pw[24 + W] = p_word<poly_word(W)>(rd + 4 * W, c2, nm2);
+    p_words32<W + 1>(ra, rb, rc, rd, pw, c2, nm2);
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <int kTiles>
+__global__ void __launch_bounds__(Cfg<kTiles>::kThreads, Cfg<kTiles>::kMinBlocks)
     icl_attention_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const KParams p) {
+  using C = Cfg<kTiles>;
+  constexpr int kSoftmaxWarps = C::kSoftmaxWarps;
+  constexpr int kProducerWarp = C::kProducerWarp;
+  constexpr int kMmaWarp = C::kMmaWarp;
+  constexpr int kThreads = C::kThreads;
+  constexpr uint32_t kTmemCols = C::kTmemCols;
+  (void)kSoftmaxWarps;
   extern __shared__ uint8_t smem_raw[];
-  Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem<kTiles>& s =
+      *reinterpret_cast<Smem<kTiles>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const volatile uint32_t* abort_flag = &s.abort_flag;
 
   const int warp = threadIdx.x >> 5;
@@ -270,14 +294,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t a0 = smem_u32(s.q[t]), b0 = smem_u32(s.k[st]);
 #pragma unroll
         for (int ks = 0; ks < kHeadDim / 32; ++ks)
-          mma_e4m3_ss(tmem + s_col(t), smem_desc_kmajor(a0 + 32 * ks, 512, kSwizzle64B),
+          mma_e4m3_ss(tmem + s_col<kTiles>(t), smem_desc_kmajor(a0 + 32 * ks, 512, kSwizzle64B),
                       smem_desc_kmajor(b0 + 32 * ks, 512, kSwizzle64B), idesc_s, ks > 0);
       };
       auto issue_pv = [&](int t, int st, bool acc) {
         const uint32_t b0 = smem_u32(s.v[st]);
 #pragma unroll
         for (int ks = 0; ks < kKvTile / 32; ++ks)
-          mma_e4m3_ts(tmem + o_col(t), tmem + p_col(t) + 8 * ks, smem_desc_kmajor(b0 + 32 * ks, 1024, kSwizzle128B),
+          mma_e4m3_ts(tmem + o_col<kTiles>(t), tmem + p_col<kTiles>(t) + 8 * ks, smem_desc_kmajor(b0 + 32 * ks, 1024, kSwizzle128B),
                       idesc_o, (acc || ks > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(&s.q_full, 0, abort_flag, kWaitLimit);
@@ -312,6 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
+#pragma unroll
         for (int t = 0; t < kTiles; ++t) {
           if (more) {
             if (!mbar_wait(&s.s_free[t], it & 1, abort_flag, kWaitLimit)) {
@@ -343,9 +368,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int t = warp >> 2;   // query tile
     const int wq = warp & 3;   // TMEM lane quadrant
     const uint32_t lane_base = static_cast<uint32_t>(32 * wq) << 16;
-    const uint32_t t_s = tmem + lane_base + s_col(t);
-    const uint32_t t_p = tmem + lane_base + p_col(t);
-    const uint32_t t_o = tmem + lane_base + o_col(t);
+    const uint32_t t_s = tmem + lane_base + s_col<kTiles>(t);
+    const uint32_t t_p = tmem + lane_base + p_col<kTiles>(t);
+    const uint32_t t_o = tmem + lane_base + o_col<kTiles>(t);
     const float s_q = __ldg(p.scales + bh);
     const float s_k = __ldg(p.scales + p.BH + bh);
     const float s_v = __ldg(p.scales + 2 * p.BH + bh);
@@ -406,14 +431,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P = 2^(fma(z, c2, -m2)) in (0, 1] -> e4m3, four codes per 32-bit TMEM column
       const float nm2 = -m2_new;
       {
-        uint32_t pw[16];
-        p_words<0>(ra, rb, pw, c2, nm2);
-        tmem_st_32x32b_x16(t_p, pw);
-      }
-      {
-        uint32_t pw[16];
-        p_words<0>(rc, rd, pw, c2, nm2);
-        tmem_st_32x32b_x16(t_p + 16, pw);
+        // all 32 words first, one store: the store's memory clobber would
+        // otherwise keep the scheduler from interleaving the two halves
+        uint32_t pw[32];
+        p_words32<0>(ra, rb, rc, rd, pw, c2, nm2);
+        tmem_st_32x32b_x32(t_p, pw);
       }
       if (it > 0 && __any_sync(0xffffffffu, up)) {
         // O and its row sum were accumulated against the old max: rescale (after
@@ -578,6 +600,20 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <int kTiles>
+cudaError_t launch_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, KParams p, int64_t BH,
+                          cudaStream_t st) {
+  p.n_pairs = (p.T + kTiles * kQTile - 1) / (kTiles * kQTile);
+  const size_t smem = sizeof(Smem<kTiles>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(icl_attention_kernel<kTiles>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int64_t grid = p.n_pairs * p.n_splits * BH;
+  if (grid == 0) return cudaSuccess;
+  icl_attention_kernel<kTiles><<<static_cast<unsigned>(grid), Cfg<kTiles>::kThreads, smem, st>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8t, const AttnArgs& a,
@@ -596,7 +632,6 @@ cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t
   p.H = a.H;
   p.T = a.T;
   p.N = a.N;
-  p.n_pairs = (a.T + kTiles * kQTile - 1) / (kTiles * kQTile);
   p.n_splits = a.partial ? a.n_splits : 1;
   p.split_keys = a.split_keys;
   p.partial = a.partial ? 1 : 0;
@@ -605,14 +640,9 @@ cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t
   p.part_acc = a.part_acc;
   p.part_ml = a.part_ml;
   p.err = a.err;
-  const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(icl_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  const int64_t grid = p.n_pairs * p.n_splits * BH;
-  if (grid == 0) return cudaSuccess;
-  icl_attention_kernel<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(tq, tk, tv, p);
-  return cudaGetLastError();
+  // at most 128 rows (small prediction batches): one query tile per CTA, two CTAs per SM
+  if (a.T <= kQTile) return launch_kernel<1>(tq, tk, tv, p, BH, st);
+  return launch_kernel<2>(tq, tk, tv, p, BH, st);
 }
 
 cudaError_t launch_splitkv_reduce(const AttnArgs& a, cudaStream_t st) {
