@@ -376,6 +376,8 @@ __global__ void __launch_bounds__(Cfg<kTiles>::kThreads, Cfg<kTiles>::kMinBlocks
     const float s_v = __ldg(p.scales + 2 * p.BH + bh);
     // c2 = s_q * s_k * log2(e) / sqrt(64): logits in base-2 units per raw z
     const float c2 = __fmul_rn(__fmul_rn(s_q, s_k), 0.18033688011112042f);
+    // does this warp own any row below T? (only the 1-tile kernel skips warps)
+    const bool warp_rows = kTiles == 1 ? (row0 + 32 * wq < p.T) : true;
     float m_run = -INFINITY;  // running max of raw z
     float m2 = -INFINITY;     // fp32(m_run * c2)
     bool ok = true;
@@ -387,6 +389,26 @@ __global__ void __launch_bounds__(Cfg<kTiles>::kThreads, Cfg<kTiles>::kMinBlocks
         break;
       }
       tc_fence_after();
+      if constexpr (kTiles == 1) {
+        if (!warp_rows) {
+          // Small batches: every row of this warp lies past the last query
+          // row, so skip the logits but keep the barrier protocol in step --
+          // the p_full arrival waits, like the other warps' P stores, for the
+          // previous P V (o_ready), so it can never count toward an older phase.
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s.s_free[t]);
+          if (it > 0) {
+            ok = mbar_wait(&s.o_ready[t], (it - 1) & 1, abort_flag, kWaitLimit);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) {
+              if (lane == 0) raise_abort(s, p.err, kErrTimeoutO);
+              break;
+            }
+          }
+          if (lane == 0) mbar_arrive(&s.p_full[t]);
+          continue;
+        }
+      }
       const int64_t nvalid = kv_end - (kv_begin + (int64_t)it * kKvTile);
       const bool ragged = nvalid < kKvTile;
       // one read of the 128 logits: four loads in flight, one wait
