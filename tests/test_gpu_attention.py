@@ -106,3 +106,9 @@ def test_layer_512k_sampled(cuda_lib, orc):
     w = WORKLOADS["icl_n512k_m1k_h8"]
     inp = make_inputs(w)
     _layer_case(cuda_lib, orc, inp, rows=_sample_rows(w.n_ctx, w.n_query, 64, 128, 4), report="512K")
+
+
+def test_layer_max_heads(cuda_lib, orc):
+    """128 heads (the largest the ABI accepts), small context."""
+    inp = make_inputs(WORKLOADS["icl_n1k_m128_h4"], n_ctx=200, n_query=30, heads=128)
+    _layer_case(cuda_lib, orc, inp, report="H128")

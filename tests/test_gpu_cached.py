@@ -62,3 +62,20 @@ def test_cached_512k_full_size(cuda_lib, orc):
     rows = np.sort(np.random.default_rng(5).choice(w.n_query, 96, replace=False)).astype(np.int64)
     _, o, allow = _oracle_cached(orc, inp, inp["queries"], rows=rows)
     print("\ncached 512K:", gate(full[:, rows], o, allow, "cached 512K"))
+
+
+def test_cached_batch2_gated_queries(cuda_lib, orc):
+    """B = 2 (per-(b, h) scales) and GatedLogScale on the prediction queries."""
+    B, N, M, H = 2, 17000, 40, 3
+    inp = make_inputs(WORKLOADS["cached_n512k_m1k_h8"], n_ctx=N, n_query=M, heads=H, batch=B)
+    cache = _fit(cuda_lib, inp)
+    rng = np.random.default_rng(7)
+    g_q = (rng.standard_normal((B, M, H)) * 1.5).astype(np.float16)
+    out = cuda_lib.cached_attention(dev(inp["queries"]), cache, dev(inp["c_h"]), dev(g_q))
+    torch.cuda.synchronize()
+    qs = orc.qscale(inp["q"], N, inp["c_h"])
+    s_q, s_k, s_v = (orc.context_scales(x, N) for x in (qs, inp["k"], inp["v"]))
+    qq = orc.quantize(orc.qscale(inp["queries"], N, inp["c_h"], g_q), s_q)
+    _, o, allow = orc.attention(qq, orc.quantize(inp["k"], s_k), orc.quantize(inp["v"], s_v), s_q, s_k, s_v,
+                                split=orc.SPLIT_KEYS, delta=DELTA)
+    print("\ncached B2 gated:", gate(out, o, allow, "cached B2 gated"))
