@@ -20,11 +20,10 @@ STATUS_NAMES = {0: "SDM_OK", 1: "SDM_ERR_INVALID_ARG", 2: "SDM_ERR_UNSUPPORTED",
                 7: "SDM_ERR_CUDA"}
 OP_QUANTIZE_CONTEXT, OP_ICL_ATTENTION, OP_CACHED_ATTENTION = 0, 1, 2
 KV_TILE = 128
-SPLIT_KEYS = 16384
 HEAD_DIM = 64
 
 # Every symbol the header declares (checked by the ABI tests).
-EXPORTS = ("sdm_status_string", "sdm_version", "sdm_cache_layout", "sdm_workspace_size", "sdm_qscale_fused",
+EXPORTS = ("sdm_status_string", "sdm_version", "sdm_split_keys", "sdm_cache_layout", "sdm_workspace_size", "sdm_qscale_fused",
            "sdm_fp8_quantize_context", "sdm_fp8_quantize_context_noalloc", "sdm_fp8_attention", "sdm_icl_attention",
            "sdm_cached_attention", "sdm_sync_status", "sdm_selftest_wait_timeout")
 NOALLOC_MAX_BATCH_HEADS = 4096
@@ -59,6 +58,8 @@ def lib() -> ctypes.CDLL:
         L.sdm_status_string.argtypes = [ctypes.c_int]
         L.sdm_version.restype = _I32
         L.sdm_version.argtypes = []
+        L.sdm_split_keys.restype = _I64
+        L.sdm_split_keys.argtypes = [_I64]
         L.sdm_cache_layout.restype = ctypes.c_int
         L.sdm_cache_layout.argtypes = [_I32, _I64, _I32, _I32, ctypes.POINTER(_SZ), ctypes.POINTER(_SZ),
                                        ctypes.POINTER(_SZ), ctypes.POINTER(_I64)]
@@ -121,6 +122,11 @@ def _want(t: torch.Tensor, dtype: torch.dtype, name: str, ndim: int) -> None:
 
 def workspace_size(op: int, batch: int, n_ctx: int, n_query: int, heads: int, keep_cache: bool = True) -> int:
     return int(lib().sdm_workspace_size(op, batch, n_ctx, n_query, heads, HEAD_DIM, 1 if keep_cache else 0))
+
+
+def split_keys(n_ctx: int) -> int:
+    """Keys per split-KV chunk of cached prediction for an n_ctx-key context."""
+    return int(lib().sdm_split_keys(int(n_ctx)))
 
 
 def new_workspace(nbytes: int, device) -> torch.Tensor:

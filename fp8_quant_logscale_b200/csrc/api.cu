@@ -79,7 +79,10 @@ struct WsLayout {
   size_t amax = 0, gate_w = 0, q8 = 0, k8 = 0, v8t = 0, scales = 0, part_acc = 0, part_ml = 0, total = 0;
 };
 
-int64_t n_splits_for(int64_t n_ctx) { return (n_ctx + kSplitKeys - 1) / kSplitKeys; }
+int64_t n_splits_for(int64_t n_ctx) {
+  const int64_t len = split_keys_for(n_ctx);
+  return (n_ctx + len - 1) / len;
+}
 
 WsLayout ws_layout(sdm_op op, int32_t B, int64_t N, int64_t M, int32_t H, int32_t keep_cache) {
   WsLayout w;
@@ -206,6 +209,8 @@ const char* sdm_status_string(sdm_status s) {
 
 int32_t sdm_version(void) { return 100; }
 
+int64_t sdm_split_keys(int64_t n_ctx) { return n_ctx < 1 ? 0 : split_keys_for(n_ctx); }
+
 sdm_status sdm_cache_layout(int32_t B, int64_t N, int32_t H, int32_t d, size_t* k8_bytes, size_t* v8t_bytes,
                             size_t* scales_bytes, int64_t* ld_v) {
   SDM_TRY(check_shape(B, N, 0, H, d));
@@ -292,7 +297,7 @@ sdm_status sdm_fp8_attention(const uint8_t* q8, int32_t B, int64_t rows, const s
   a.scales = cache->scales;
   a.partial = split != 0;
   a.n_splits = split ? n_splits_for(cache->n_ctx) : 1;
-  a.split_keys = kSplitKeys;
+  a.split_keys = split_keys_for(cache->n_ctx);
   a.out = reinterpret_cast<__half*>(out);
   a.part_acc = split ? reinterpret_cast<float*>(base + w.part_acc) : nullptr;
   a.part_ml = split ? reinterpret_cast<float*>(base + w.part_ml) : nullptr;
@@ -356,7 +361,7 @@ sdm_status sdm_icl_attention(const void* q, const void* k, const void* v, int32_
   a.scales = c->scales;
   a.partial = false;
   a.n_splits = 1;
-  a.split_keys = kSplitKeys;
+  a.split_keys = split_keys_for(N);
   a.out = reinterpret_cast<__half*>(out);
   a.part_acc = nullptr;
   a.part_ml = nullptr;
@@ -402,7 +407,7 @@ sdm_status sdm_cached_attention(const void* q, int32_t B, int64_t M, int32_t H, 
   a.scales = cache->scales;
   a.partial = true;
   a.n_splits = n_splits_for(N);
-  a.split_keys = kSplitKeys;
+  a.split_keys = split_keys_for(N);
   a.out = reinterpret_cast<__half*>(out);
   a.part_acc = reinterpret_cast<float*>(base + w.part_acc);
   a.part_ml = reinterpret_cast<float*>(base + w.part_ml);

@@ -11,7 +11,14 @@ namespace sdm {
 constexpr int kHeadDim = 64;   // the only head dimension the kernels are built for
 constexpr int kKvTile = 128;   // keys per online-softmax block (one tcgen05 N=128 tile)
 constexpr int kQTile = 128;    // query rows per tensor-core tile (M=128)
-constexpr int64_t kSplitKeys = 16384;  // cached prediction: keys per split-KV chunk
+// Cached prediction: keys per split-KV chunk, a function of the context length
+// alone (so a query's result never depends on the batch it came in): about 32
+// chunks, each a multiple of 128 keys, between 1024 and 16384 keys.
+constexpr int64_t kSplitMin = 1024, kSplitMax = 16384, kSplitTarget = 32;
+inline int64_t split_keys_for(int64_t n_ctx) {
+  const int64_t per = (n_ctx + kSplitTarget * kKvTile - 1) / (kSplitTarget * kKvTile) * kKvTile;
+  return per < kSplitMin ? kSplitMin : (per > kSplitMax ? kSplitMax : per);
+}
 
 // Query-scaling parameters shared by the elementwise kernels.
 struct QScale {

@@ -66,11 +66,9 @@ typedef enum {
   SDM_OP_CACHED_ATTENTION = 2
 } sdm_op;
 
-/* Keys per online-softmax block and per cached-prediction split-KV chunk.
- * The chunk boundaries of the cached path depend on the context length only,
- * so a query's cached prediction does not depend on how queries are batched. */
+/* Keys per online-softmax block (blocks start at key 0, or at the chunk start
+ * on the cached path). */
 #define SDM_KV_TILE 128
-#define SDM_SPLIT_KEYS 16384
 
 /*
  * FP8 K/V cache: the fitted state that cached prediction reads (the analogue
@@ -101,6 +99,14 @@ const char* sdm_status_string(sdm_status status);
 
 /* Library version as major*10000 + minor*100 + patch. */
 int32_t sdm_version(void);
+
+/*
+ * Keys per split-KV chunk of cached prediction for a context of n_ctx keys:
+ * min(16384, max(1024, 128 * ceil(n_ctx / 4096))) -- about 32 chunks.  It
+ * depends on the context length only, so a query's cached prediction does not
+ * depend on how the queries are batched.  Returns 0 for n_ctx < 1.
+ */
+int64_t sdm_split_keys(int64_t n_ctx);
 
 /*
  * Byte sizes of the three cache buffers for B x N x H x d, and ld_v.
@@ -161,8 +167,8 @@ sdm_status sdm_fp8_quantize_context(const void* q_scaled, const void* k, const v
  *   q8     [B][H][rows][d] e4m3
  *   cache  filled FP8 cache (k8, v8t, scales)
  *   out    [B][rows][H][d] fp16
- *   split  0: one pass over all keys; 1: split-KV in SDM_SPLIT_KEYS chunks
- *          combined in chunk order (the cached-prediction arithmetic)
+ *   split  0: one pass over all keys; 1: split-KV in sdm_split_keys(N)-key
+ *          chunks combined in chunk order (the cached-prediction arithmetic)
  *   ws     >= sdm_workspace_size(SDM_OP_CACHED_ATTENTION, B, N, rows, ...)
  */
 sdm_status sdm_fp8_attention(const uint8_t* q8, int32_t batch, int64_t rows, const sdm_fp8_cache* cache, void* out,
@@ -190,7 +196,7 @@ sdm_status sdm_icl_attention(const void* q, const void* k, const void* v, int32_
  * Step 4 -- cached prediction ("model.predict(queries)" after "model.fit" on
  * "[FP8 3/4] ...").  The M query rows are query-scaled with n = cache->n_ctx,
  * quantised with the cache's context-derived s_q, and attend to the cache's
- * keys with split-KV (SDM_SPLIT_KEYS-key chunks, a fixed-order combine), so a
+ * keys with split-KV (sdm_split_keys(N)-key chunks, a fixed-order combine), so a
  * query's output is identical however the queries are batched.
  *   q    [B][M][H][d] fp16 raw;  gate [B][M][H] fp16 or NULL;  c_h [H] fp32
  *   out  [B][M][H][d] fp16

@@ -24,10 +24,16 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 
 # KV tile (online-softmax block) and cached-prediction split length that the
 # layer is defined with.  These are algorithm parameters, restated here on the
-# oracle side from the layer's specification (128-key tiles; the cached path
-# cuts the keys into 16384-key chunks whose boundaries depend on N only).
+# oracle side from the layer's specification: 128-key tiles; the cached path
+# cuts the keys into chunks whose length depends on N only -- about 32 chunks,
+# each a multiple of 128 keys, clamped to [1024, 16384].
 KV_TILE = 128
-SPLIT_KEYS = 16384
+
+
+def split_keys(n_ctx: int) -> int:
+    """Chunk length of the cached-prediction split for an n_ctx-key context."""
+    per = -(-n_ctx // (32 * KV_TILE)) * KV_TILE
+    return min(16384, max(1024, per))
 
 
 def build(force: bool = False) -> str:

@@ -76,3 +76,11 @@ def test_shape_errors_before_any_cuda_call(L):
 def test_no_device_reports_cuda_error(L):
     # valid shapes, no GPU: the device query fails and nothing is launched
     assert L.sdm_qscale_fused(None, None, 1, 10, 4, 64, 10, None, None, None) == 7
+
+
+def test_split_length_rule_matches_the_oracle(L, orc):
+    """Cached prediction's chunk length is a function of N alone, the same on both sides."""
+    for n in [1, 100, 1024, 4096, 4097, 16384, 20000, 131072, 131073, 524288, 1 << 22, 1 << 26]:
+        assert L.sdm_split_keys(n) == orc.split_keys(n), n
+    assert L.sdm_split_keys(524288) == 16384 and L.sdm_split_keys(16384) == 1024
+    assert L.sdm_split_keys(0) == 0

@@ -23,7 +23,7 @@ def _oracle_cached(orc, inp, queries, rows=None):
     s_q, s_k, s_v = (orc.context_scales(x, N) for x in (qs, inp["k"], inp["v"]))
     k8, v8 = orc.quantize(inp["k"], s_k), orc.quantize(inp["v"], s_v)
     qq = orc.quantize(orc.qscale(queries, N, inp["c_h"]), s_q)
-    return orc.attention(qq, k8, v8, s_q, s_k, s_v, rows=rows, split=orc.SPLIT_KEYS, delta=DELTA)
+    return orc.attention(qq, k8, v8, s_q, s_k, s_v, rows=rows, split=orc.split_keys(N), delta=DELTA)
 
 
 @pytest.mark.parametrize("N,M,H", [(20000, 300, 3), (16384, 64, 8), (1000, 1, 2), (33000, 129, 4)])
@@ -77,5 +77,5 @@ def test_cached_batch2_gated_queries(cuda_lib, orc):
     s_q, s_k, s_v = (orc.context_scales(x, N) for x in (qs, inp["k"], inp["v"]))
     qq = orc.quantize(orc.qscale(inp["queries"], N, inp["c_h"], g_q), s_q)
     _, o, allow = orc.attention(qq, orc.quantize(inp["k"], s_k), orc.quantize(inp["v"], s_v), s_q, s_k, s_v,
-                                split=orc.SPLIT_KEYS, delta=DELTA)
+                                split=orc.split_keys(N), delta=DELTA)
     print("\ncached B2 gated:", gate(out, o, allow, "cached B2 gated"))
