@@ -156,12 +156,14 @@ class FP8Cache:
         _check(lib().sdm_cache_layout(batch, n_ctx, heads, HEAD_DIM, ctypes.byref(kb), ctypes.byref(vb),
                                       ctypes.byref(sb), ctypes.byref(ld)), "sdm_cache_layout")
         device = torch.device(device)
+        if device.index is None:
+            device = torch.device("cuda", torch.cuda.current_device())
         self.k8 = torch.empty((batch, heads, n_ctx, HEAD_DIM), dtype=torch.uint8, device=device)
         self.v8t = torch.empty((batch, heads, HEAD_DIM, ld.value), dtype=torch.uint8, device=device)
         self.scales = torch.empty((3, batch, heads), dtype=torch.float32, device=device)
         assert self.k8.numel() == kb.value and self.v8t.numel() == vb.value and self.scales.numel() * 4 == sb.value
         self.struct = CacheStruct(self.k8.data_ptr(), self.v8t.data_ptr(), self.scales.data_ptr(), n_ctx, ld.value,
-                                  batch, heads, HEAD_DIM, device.index if device.index is not None else 0, 0)
+                                  batch, heads, HEAD_DIM, device.index, 0)
 
     @property
     def filled(self) -> bool:
