@@ -440,23 +440,22 @@ __global__ void __launch_bounds__(Cfg<kTiles>::kThreads, Cfg<kTiles>::kMinBlocks
       const float mt = max3(mx0, mx1, fmaxf(mx2, mx3));
       const bool up = mt > m_run;
       const float m2_new = up ? __fmul_rn(mt, c2) : m2;
-      // the previous P_t V must be done before P_t is overwritten and O_t rescaled
-      if (it > 0) {
-        ok = mbar_wait(&s.o_ready[t], (it - 1) & 1, abort_flag, kWaitLimit);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) {
-          if (lane == 0) raise_abort(s, p.err, kErrTimeoutO);
-          break;
-        }
-        tc_fence_after();
-      }
       // P = 2^(fma(z, c2, -m2)) in (0, 1] -> e4m3, four codes per 32-bit TMEM column
       const float nm2 = -m2_new;
       {
-        // all 32 words first, one store: the store's memory clobber would
-        // otherwise keep the scheduler from interleaving the two halves
         uint32_t pw[32];
         p_words32<0>(ra, rb, rc, rd, pw, c2, nm2);
+        // the previous P_t V must be done before P_t is overwritten and O_t
+        // rescaled; waiting only now gives that MMA the whole P computation
+        if (it > 0) {
+          ok = mbar_wait(&s.o_ready[t], (it - 1) & 1, abort_flag, kWaitLimit);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) {
+            if (lane == 0) raise_abort(s, p.err, kErrTimeoutO);
+            break;
+          }
+          tc_fence_after();
+        }
         tmem_st_32x32b_x32(t_p, pw);
       }
       if (it > 0 && __any_sync(0xffffffffu, up)) {
