@@ -41,7 +41,7 @@ BF16_NOMINAL_TFLOPS = 2250.0
 # 512K workload, from a one-pass ncu capture (profiles/icl_attention_kernel_n512k_dram.md).
 # Valid only for the kernel source it was taken on: any change to these files
 # makes the bench report null until a new capture is recorded here.
-ATTN_TRAFFIC_SOURCES = ("attention.cu", "ptx.cuh", "exp2_poly.cuh", "kernels.cuh")
+ATTN_TRAFFIC_SOURCES = ("attention.cu", "ptx.cuh", "exp2_poly.cuh", "kernels.cuh", "softmax.cuh")
 ATTN_TRAFFIC = {"source_sha256": "143dadd20328697008c365ba22efb292ff88a7395e04e94df6dd12b4d9300425",
                 "bytes": 5.93e9 + 592.26e6}
 
