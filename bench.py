@@ -42,8 +42,8 @@ BF16_NOMINAL_TFLOPS = 2250.0
 # Valid only for the kernel source it was taken on: any change to these files
 # makes the bench report null until a new capture is recorded here.
 ATTN_TRAFFIC_SOURCES = ("attention.cu", "ptx.cuh", "exp2_poly.cuh", "kernels.cuh", "softmax.cuh")
-ATTN_TRAFFIC = {"source_sha256": "143dadd20328697008c365ba22efb292ff88a7395e04e94df6dd12b4d9300425",
-                "bytes": 5.93e9 + 592.26e6}
+ATTN_TRAFFIC = {"source_sha256": "5d31a51a6a85efefca0cacd5da144e97d506db923f9cc373bf368c79670f2846",
+                "bytes": 6.39e9 + 684.83e6}
 
 
 def attention_source_sha256() -> str:
@@ -201,6 +201,7 @@ def run_ours(args):
     cache = sdm.FP8Cache(B, N, H, device)
     ws_icl = sdm.new_workspace(sdm.workspace_size(binding.OP_ICL_ATTENTION, B, N, M, H, keep_cache=True), device)
     ws_c = sdm.new_workspace(sdm.workspace_size(binding.OP_CACHED_ATTENTION, B, N, Mq, H), device)
+    ws_h = sdm.new_workspace(sdm.workspace_size(binding.OP_ICL_ATTENTION_F16, B, N, M, H), device)
     stream = torch.cuda.current_stream(device)
 
     def step():
@@ -367,10 +368,12 @@ def run_per_kernel(args):
     queries = q[:, :Mq].contiguous()
     pred = torch.empty_like(queries)
     ws_c = sdm.new_workspace(sdm.workspace_size(binding.OP_CACHED_ATTENTION, B, N, Mq, H), device)
+    ws_h = sdm.new_workspace(sdm.workspace_size(binding.OP_ICL_ATTENTION_F16, B, N, M, H), device)
     stream = torch.cuda.current_stream(device)
     peaks = measured_peaks() or {"hbm_gbs": 6650.0, "bf16_tflops_sustained": 1400.0}
     hbm = peaks["hbm_gbs"]
-    fp8 = peaks["bf16_tflops_sustained"] * FP8_NOMINAL_TFLOPS / BF16_NOMINAL_TFLOPS
+    f16 = peaks["bf16_tflops_sustained"]  # fp16 and bf16 share the tensor-core rate
+    fp8 = f16 * FP8_NOMINAL_TFLOPS / BF16_NOMINAL_TFLOPS
     el = lambda rows: B * rows * H * 64
     steps = [
         # name, call, algorithmic bytes, flops
@@ -386,6 +389,10 @@ def run_per_kernel(args):
         ("a4 cached prediction, 1024 queries (sdm_cached_attention)",
          lambda: sdm.cached_attention(queries, cache, c_h, gate=None, out=pred, ws=ws_c),
          2 * el(Mq) + 2 * el(N) + 2 * el(Mq), attn_flops(Mq, N, H)),
+        ("a5 fp16 attention, query scaling included (sdm_icl_attention_f16)",
+         lambda: sdm.icl_attention_f16(q, k, v, N, c_h, gate, out=out, ws=ws_h),
+         # q -> q' (4 B), V -> V^T (4 B), then q', K, V^T read and O written (2 B each)
+         4 * el(T) + 4 * el(N) + 2 * el(T) + 4 * el(N) + 2 * el(T), attn_flops(T, N, H)),
     ]
     # a filled cache and Q8 for the attention steps
     q8.copy_(sdm.fp8_quantize_context(sdm.qscale_fused(q, c_h, N, gate), k, v, N, cache=cache)[0])
@@ -403,7 +410,9 @@ def run_per_kernel(args):
         line = {"step": name, "workload": w.name, "ms": ms, "bytes": nbytes,
                 "gbs": nbytes / (ms * 1e-3) / 1e9, "frac_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm}
         if flops:
-            line.update({"tflops": flops / (ms * 1e-3) / 1e12, "frac_fp8": flops / (ms * 1e-3) / 1e12 / fp8})
+            tf = flops / (ms * 1e-3) / 1e12
+            line.update({"tflops": tf, "frac_f16" if name.startswith("a5") else "frac_fp8":
+                         tf / (f16 if name.startswith("a5") else fp8)})
         print(json.dumps(line), flush=True)
 
 

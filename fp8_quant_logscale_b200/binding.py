@@ -18,14 +18,16 @@ SDM_OK = 0
 STATUS_NAMES = {0: "SDM_OK", 1: "SDM_ERR_INVALID_ARG", 2: "SDM_ERR_UNSUPPORTED", 3: "SDM_ERR_WORKSPACE",
                 4: "SDM_ERR_DEVICE_MISMATCH", 5: "SDM_ERR_CACHE_MISMATCH", 6: "SDM_ERR_TIMEOUT",
                 7: "SDM_ERR_CUDA"}
-OP_QUANTIZE_CONTEXT, OP_ICL_ATTENTION, OP_CACHED_ATTENTION = 0, 1, 2
+OP_QUANTIZE_CONTEXT, OP_ICL_ATTENTION, OP_CACHED_ATTENTION, OP_ICL_ATTENTION_F16 = 0, 1, 2, 3
+FP8_MIN_CONTEXT = 8192
 KV_TILE = 128
 HEAD_DIM = 64
 
 # Every symbol the header declares (checked by the ABI tests).
 EXPORTS = ("sdm_status_string", "sdm_version", "sdm_split_keys", "sdm_cache_layout", "sdm_workspace_size", "sdm_qscale_fused",
            "sdm_fp8_quantize_context", "sdm_fp8_quantize_context_noalloc", "sdm_fp8_attention", "sdm_icl_attention",
-           "sdm_cached_attention", "sdm_sync_status", "sdm_selftest_wait_timeout")
+           "sdm_cached_attention", "sdm_fp8_eligible", "sdm_icl_attention_f16", "sdm_sync_status",
+           "sdm_selftest_wait_timeout")
 NOALLOC_MAX_BATCH_HEADS = 4096
 
 
@@ -81,6 +83,10 @@ def lib() -> ctypes.CDLL:
         L.sdm_cached_attention.restype = ctypes.c_int
         L.sdm_cached_attention.argtypes = [_P, _I32, _I64, _I32, _I32, ctypes.POINTER(CacheStruct), _P, _P, _P,
                                            _P, _SZ, _P]
+        L.sdm_fp8_eligible.restype = _I32
+        L.sdm_fp8_eligible.argtypes = [_I64, _I32]
+        L.sdm_icl_attention_f16.restype = ctypes.c_int
+        L.sdm_icl_attention_f16.argtypes = [_P, _P, _P, _I32, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _SZ, _P]
         L.sdm_selftest_wait_timeout.restype = ctypes.c_int
         L.sdm_selftest_wait_timeout.argtypes = [_P, _I64, _P]
         L.sdm_sync_status.restype = ctypes.c_int
@@ -288,3 +294,48 @@ def cached_attention(q: torch.Tensor, cache: FP8Cache, c_h: torch.Tensor, gate: 
         _check(lib().sdm_cached_attention(_ptr(q), B, M, H, d, ctypes.byref(cache.struct), _ptr(c_h), _ptr(gate),
                                           _ptr(out), _ptr(ws), ws.numel(), _stream(dev)), "sdm_cached_attention")
     return out
+
+
+def fp8_eligible(n_unmasked_ctx: int, final_layer: bool = False) -> bool:
+    """The precision rule: FP8 attention only on a non-final ICL layer above 8,192 unmasked context rows."""
+    return bool(lib().sdm_fp8_eligible(int(n_unmasked_ctx), 1 if final_layer else 0))
+
+
+def icl_attention_f16(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_ctx: int, c_h: torch.Tensor | None,
+                      gate: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                      ws: torch.Tensor | None = None) -> torch.Tensor:
+    """Normal-precision layer call: q [B,T,H,64] raw fp16, k/v [B,N,H,64] fp16 -> out [B,T,H,64] fp16.
+
+    c_h None: no query scaling (q is used as given; gate must be None).
+    """
+    _want(q, torch.float16, "q", 4)
+    _want(k, torch.float16, "k", 4)
+    _want(v, torch.float16, "v", 4)
+    if c_h is not None:
+        _want(c_h, torch.float32, "c_h", 1)
+    if gate is not None:
+        _want(gate, torch.float16, "gate", 3)
+    B, T, H, d = q.shape
+    M = T - n_ctx
+    dev = q.device
+    out = torch.empty_like(q) if out is None else out
+    need = workspace_size(OP_ICL_ATTENTION_F16, B, n_ctx, M, H)
+    ws = new_workspace(need, dev) if ws is None else ws
+    with torch.cuda.device(dev):
+        _check(lib().sdm_icl_attention_f16(_ptr(q), _ptr(k), _ptr(v), B, n_ctx, M, H, d, _ptr(c_h), _ptr(gate),
+                                           _ptr(out), _ptr(ws), ws.numel(), _stream(dev)), "sdm_icl_attention_f16")
+    return out
+
+
+def icl_layer(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_ctx: int, c_h: torch.Tensor,
+              gate: torch.Tensor | None = None, final_layer: bool = False, cache: FP8Cache | None = None,
+              out: torch.Tensor | None = None) -> torch.Tensor:
+    """One ICL attention layer with the precision rule applied: FP8 (icl_attention) when
+    fp8_eligible(n_ctx, final_layer), else normal precision (icl_attention_f16).  A cache
+    can only be filled on the FP8 path."""
+    if fp8_eligible(n_ctx, final_layer):
+        return icl_attention(q, k, v, n_ctx, c_h, gate=gate, cache=cache, out=out)
+    if cache is not None:
+        raise ValueError("an FP8 cache is filled only by an FP8-eligible layer "
+                         f"(n_ctx={n_ctx}, final_layer={final_layer})")
+    return icl_attention_f16(q, k, v, n_ctx, c_h, gate=gate, out=out)

@@ -77,6 +77,7 @@ sdm_status check_tensor(const void* p, int dev) {
 // Workspace carve-up.  Offsets are 1 KB aligned; the error word sits at 0.
 struct WsLayout {
   size_t amax = 0, gate_w = 0, q8 = 0, k8 = 0, v8t = 0, scales = 0, part_acc = 0, part_ml = 0, total = 0;
+  size_t q16 = 0, vt16 = 0;  // normal-precision path: q' and V^T in fp16
 };
 
 int64_t n_splits_for(int64_t n_ctx) {
@@ -88,6 +89,15 @@ WsLayout ws_layout(sdm_op op, int32_t B, int64_t N, int64_t M, int32_t H, int32_
   WsLayout w;
   const size_t BH = (size_t)B * H;
   size_t off = kErrBytes;
+  if (op == SDM_OP_ICL_ATTENTION_F16) {
+    const int64_t ld = round_up(N, kKvTile);
+    w.q16 = off;
+    off = align_up(off + BH * (size_t)(N + M) * kHeadDim * sizeof(uint16_t), kAlign);
+    w.vt16 = off;
+    off = align_up(off + BH * kHeadDim * (size_t)ld * sizeof(uint16_t), kAlign);
+    w.total = off;
+    return w;
+  }
   w.amax = off;
   off = align_up(off + 3 * BH * sizeof(uint32_t), kAlign);
   if (op == SDM_OP_QUANTIZE_CONTEXT) {
@@ -224,7 +234,9 @@ sdm_status sdm_cache_layout(int32_t B, int64_t N, int32_t H, int32_t d, size_t* 
 }
 
 size_t sdm_workspace_size(sdm_op op, int32_t B, int64_t N, int64_t M, int32_t H, int32_t d, int32_t keep_cache) {
-  if (op != SDM_OP_QUANTIZE_CONTEXT && op != SDM_OP_ICL_ATTENTION && op != SDM_OP_CACHED_ATTENTION) return 0;
+  if (op != SDM_OP_QUANTIZE_CONTEXT && op != SDM_OP_ICL_ATTENTION && op != SDM_OP_CACHED_ATTENTION &&
+      op != SDM_OP_ICL_ATTENTION_F16)
+    return 0;
   if (check_shape(B, N, M, H, d) != SDM_OK || N < 1) return 0;
   return ws_layout(op, B, N, M, H, keep_cache).total;
 }
@@ -414,6 +426,49 @@ sdm_status sdm_cached_attention(const void* q, int32_t B, int64_t M, int32_t H, 
   a.err = reinterpret_cast<uint32_t*>(base);
   SDM_CUDA(launch_attention(q8, cache->k8, cache->v8t, a, st));
   SDM_CUDA(launch_splitkv_reduce(a, st));
+  return SDM_OK;
+}
+
+int32_t sdm_fp8_eligible(int64_t n_unmasked_ctx, int32_t final_layer) {
+  return (final_layer == 0 && n_unmasked_ctx > SDM_FP8_MIN_CONTEXT) ? 1 : 0;
+}
+
+sdm_status sdm_icl_attention_f16(const void* q, const void* k, const void* v, int32_t B, int64_t N, int64_t M,
+                                 int32_t H, int32_t d, const float* c_h, const void* gate, void* out, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  SDM_TRY(check_shape(B, N, M, H, d));
+  if (N < 1) return SDM_ERR_INVALID_ARG;
+  const int dev = current_device();
+  if (dev < 0) return SDM_ERR_CUDA;
+  SDM_TRY(check_tensor(q, dev));
+  SDM_TRY(check_tensor(k, dev));
+  SDM_TRY(check_tensor(v, dev));
+  SDM_TRY(check_tensor(out, dev));
+  if (c_h != nullptr) {
+    if (!aligned(c_h, 4)) return SDM_ERR_INVALID_ARG;
+    if (!on_device(c_h, dev)) return SDM_ERR_DEVICE_MISMATCH;
+  }
+  if (gate != nullptr) {
+    if (c_h == nullptr || !aligned(gate, 2)) return SDM_ERR_INVALID_ARG;
+    if (!on_device(gate, dev)) return SDM_ERR_DEVICE_MISMATCH;
+  }
+  const WsLayout w = ws_layout(SDM_OP_ICL_ATTENTION_F16, B, N, M, H, 0);
+  SDM_TRY(check_ws(ws, ws_bytes, w.total, dev));
+  cudaStream_t st = as_stream(stream);
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  const int64_t T = N + M;
+  const int64_t ld = round_up(N, kKvTile);
+  const __half* qs = reinterpret_cast<const __half*>(q);
+  if (c_h != nullptr) {
+    __half* q16 = reinterpret_cast<__half*>(base + w.q16);
+    SDM_CUDA(launch_qscale(qs, q16, B, T, H, make_qscale(N, c_h, gate), st));
+    qs = q16;
+  }
+  __half* vt16 = reinterpret_cast<__half*>(base + w.vt16);
+  RowsDesc dv{reinterpret_cast<const __half*>(v), B, H, N};
+  SDM_CUDA(launch_transpose_vt_f16(dv, N, vt16, ld, st));
+  SDM_CUDA(launch_attention_f16(qs, reinterpret_cast<const __half*>(k), vt16, B, T, N, H, ld,
+                                reinterpret_cast<__half*>(out), reinterpret_cast<uint32_t*>(base), st));
   return SDM_OK;
 }
 

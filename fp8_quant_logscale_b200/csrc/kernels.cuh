@@ -58,6 +58,15 @@ cudaError_t launch_quantize_rows(RowsDesc x, QScale qs, int64_t n_rows, const fl
 cudaError_t launch_quantize_vt(RowsDesc v, int64_t n_ctx, const float* scale, uint8_t* dst, int64_t ld,
                                cudaStream_t st);
 
+// fp16 transpose of V for the normal-precision attention: dst[b][h][e][ld] =
+// v[b][key][h][e] for keys [0, n_ctx), zeros in [n_ctx, round_up(n_ctx, 128)).
+cudaError_t launch_transpose_vt_f16(RowsDesc v, int64_t n_ctx, __half* dst, int64_t ld, cudaStream_t st);
+
+// fp16 attention of rows [0, T) of q_scaled [B][T][H][64] to keys [0, N) of
+// k [B][N][H][64] and vt [B][H][64][ld]; out [B][T][H][64] fp16.
+cudaError_t launch_attention_f16(const __half* q_scaled, const __half* k, const __half* vt, int32_t B, int64_t T,
+                                 int64_t N, int32_t H, int64_t ld_v, __half* out, uint32_t* err, cudaStream_t st);
+
 // ---------------------------------------------------------------- attention
 struct AttnArgs {
   int32_t B, H;

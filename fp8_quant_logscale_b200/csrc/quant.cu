@@ -290,7 +290,54 @@ __global__ void __launch_bounds__(256) quantize_vt_kernel(RowsDesc V, int64_t n_
   }
 }
 
+// One (b, h) and 128 keys per block: 16-byte row loads of V, a shared-memory
+// transpose, 32-bit stores of 64 rows (one per head element) of 128 keys.
+__global__ void __launch_bounds__(256) transpose_vt_f16_kernel(RowsDesc V, int64_t n_ctx, __half* __restrict__ dst,
+                                                               int64_t ld) {
+  __shared__ uint16_t tile[kHeadDim][kKvTile + 2];  // [e][key]; 65-word rows
+  const int H = V.H;
+  const int64_t bh = blockIdx.y;
+  const int b = static_cast<int>(bh / H), h = static_cast<int>(bh % H);
+  const int64_t r0 = (int64_t)blockIdx.x * kKvTile;
+  const int t = threadIdx.x;
+  const int j = t & 7;  // elements 8j..8j+7
+  uint4 raws[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t r = r0 + (t >> 3) + 32 * i;
+    raws[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (r < n_ctx)
+      raws[i] = __ldcs(reinterpret_cast<const uint4*>(V.x + (((int64_t)b * V.rows + r) * H + h) * kHeadDim) + j);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int rl = (t >> 3) + 32 * i;
+    const uint32_t w[4] = {raws[i].x, raws[i].y, raws[i].z, raws[i].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      tile[8 * j + 2 * e][rl] = static_cast<uint16_t>(w[e] & 0xFFFFu);
+      tile[8 * j + 2 * e + 1][rl] = static_cast<uint16_t>(w[e] >> 16);
+    }
+  }
+  __syncthreads();
+  uint32_t* out = reinterpret_cast<uint32_t*>(dst + bh * kHeadDim * ld + r0);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int c = t + 256 * i;  // 64 rows x 64 words
+    const int e = c >> 6, wd = c & 63;
+    const uint32_t lo = tile[e][2 * wd], hi = tile[e][2 * wd + 1];
+    out[(int64_t)e * (ld / 2) + wd] = lo | (hi << 16);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_transpose_vt_f16(RowsDesc v, int64_t n_ctx, __half* dst, int64_t ld, cudaStream_t st) {
+  dim3 grid(static_cast<unsigned>((n_ctx + kKvTile - 1) / kKvTile), static_cast<unsigned>(v.B * v.H));
+  if (grid.x == 0) return cudaSuccess;
+  transpose_vt_f16_kernel<<<grid, 256, 0, st>>>(v, n_ctx, dst, ld);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_qscale(const __half* q, __half* out, int32_t B, int64_t rows, int32_t H, QScale qs,
                           cudaStream_t st) {

@@ -23,12 +23,15 @@ __device__ __forceinline__ void mask_keys(uint32_t (&ra)[32], uint32_t (&rb)[32]
 // 2^t on the FMA pipe for a pair of lanes: t = j + f with j = round(t) (the
 // 1.5*2^23 rounding trick), f in [-1/2, 1/2], 2^f from the degree-4 Remez
 // polynomial of exp2_poly.cuh (relative error < 3e-6), and 2^j added to the
-// exponent field.  t is clamped at -30 first: every result below 2^-10 is an
-// e4m3 zero anyway, and the clamp keeps the exponent arithmetic in range.
+// exponent field.  t is clamped at kClamp first, which keeps the exponent
+// arithmetic in range (kClamp >= -125 gives a normal fp32 result).  The FP8
+// kernel clamps at -30: every result below 2^-10 is an e4m3 zero anyway.
+template <int kClamp = -30>
 __device__ __forceinline__ void exp2_fma2(float t0, float t1, float& p0, float& p1) {
+  static_assert(kClamp >= -125 && kClamp <= 0, "clamp keeps 2^j a normal float");
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  t0 = fmaxf(t0, -30.0f);
-  t1 = fmaxf(t1, -30.0f);
+  t0 = fmaxf(t0, static_cast<float>(kClamp));
+  t1 = fmaxf(t1, static_cast<float>(kClamp));
   float r0, r1, j0, j1, f0, f1;
   add2(r0, r1, t0, t1, kRound, kRound);
   sub2(j0, j1, r0, r1, kRound, kRound);

@@ -61,6 +61,11 @@ WORKLOADS = {
     "icl_n512k_m1k_h8": Workload(
         "icl_n512k_m1k_h8", 524288, 1024, 8, seed=4,
         description="N=524288, M=1024, H=8, d=64, fp16 N(0,1); LogScale; FP8 self + cross attention"),
+    "final_n8k_m1k_h8_gated": Workload(
+        "final_n8k_m1k_h8_gated", 8192, 1024, 8, head_factor=(0.5, 4.0), gated=True, seed=6,
+        description="N=8192, M=1024, H=8, d=64, fp16 N(0,1) scaled per (tensor, head) by U(0.5,4); "
+                    "GatedLogScale; at most 8,192 context rows (or the final layer): normal-precision fp16 "
+                    "attention"),
     "cached_n512k_m1k_h8": Workload(
         "cached_n512k_m1k_h8", 524288, 1024, 8, cached=True, seed=5,
         description="M=1024 fp16 N(0,1) queries, H=8, d=64, LogScale n=524288, against a resident FP8 "

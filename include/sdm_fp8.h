@@ -63,7 +63,8 @@ typedef enum {
 typedef enum {
   SDM_OP_QUANTIZE_CONTEXT = 0,
   SDM_OP_ICL_ATTENTION = 1,
-  SDM_OP_CACHED_ATTENTION = 2
+  SDM_OP_CACHED_ATTENTION = 2,
+  SDM_OP_ICL_ATTENTION_F16 = 3
 } sdm_op;
 
 /* Keys per online-softmax block (blocks start at key 0, or at the chunk start
@@ -207,6 +208,39 @@ sdm_status sdm_icl_attention(const void* q, const void* k, const void* v, int32_
 sdm_status sdm_cached_attention(const void* q, int32_t batch, int64_t n_query, int32_t heads, int32_t head_dim,
                                 const sdm_fp8_cache* cache, const float* c_h, const void* gate, void* out, void* ws,
                                 size_t ws_bytes, void* stream);
+
+/*
+ * Precision rule ("[FP8 3/4] Integrate FP8 attention and caching into
+ * TabICLv2", opening section): FP8 attention serves the intermediate ICL
+ * layers only, and only above 8,192 unmasked context rows; the final ICL
+ * layer and shorter contexts keep normal-precision attention.  Returns 1 when
+ * a layer with `n_unmasked_ctx` unmasked context rows (final_layer != 0 for
+ * the last ICL layer) takes sdm_icl_attention, 0 when it takes
+ * sdm_icl_attention_f16.  Pure host function; no CUDA call.
+ */
+#define SDM_FP8_MIN_CONTEXT 8192
+int32_t sdm_fp8_eligible(int64_t n_unmasked_ctx, int32_t final_layer);
+
+/*
+ * Normal-precision ICL attention: the path the precision rule keeps for the
+ * final ICL layer and for contexts of at most 8,192 rows ("[FP8 3/4] ...",
+ * opening section; the pages run it through the framework's scaled
+ * dot-product attention).  Same rows, masking and query scaling as
+ * sdm_icl_attention: out = softmax(q' k^T / sqrt(d)) v over the N context
+ * keys, with fp16 q', k, v on the tensor cores, fp32 logits and accumulation,
+ * fp16 probabilities in the P.V product, fp16 output.  No quantisation and
+ * no cache.
+ *   q     [B][T][H][d] fp16 raw, T = N + M
+ *   k, v  [B][N][H][d] fp16
+ *   c_h   [H] fp32 device: query scaling with n = N (gate [B][T][H] fp16 or
+ *         NULL); or c_h = NULL: no query scaling, q is used as given and gate
+ *         must be NULL
+ *   out   [B][T][H][d] fp16
+ *   ws    >= sdm_workspace_size(SDM_OP_ICL_ATTENTION_F16, B, N, M, H, d, 0)
+ */
+sdm_status sdm_icl_attention_f16(const void* q, const void* k, const void* v, int32_t batch, int64_t n_ctx,
+                                 int64_t n_query, int32_t heads, int32_t head_dim, const float* c_h,
+                                 const void* gate, void* out, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Step 2 without a workspace.  This entry point has no counterpart in the

@@ -84,3 +84,24 @@ def test_split_length_rule_matches_the_oracle(L, orc):
         assert L.sdm_split_keys(n) == orc.split_keys(n), n
     assert L.sdm_split_keys(524288) == 16384 and L.sdm_split_keys(16384) == 1024
     assert L.sdm_split_keys(0) == 0
+
+
+def test_precision_rule(L):
+    # FP8 only on a non-final ICL layer with more than 8,192 unmasked context rows
+    assert binding.FP8_MIN_CONTEXT == 8192
+    assert not binding.fp8_eligible(8192) and binding.fp8_eligible(8193)
+    assert not binding.fp8_eligible(1 << 20, final_layer=True)
+    assert not binding.fp8_eligible(0) and not binding.fp8_eligible(-5)
+    for n in (1, 1024, 8191, 8192, 8193, 16384, 524288):
+        for final in (0, 1):
+            assert L.sdm_fp8_eligible(n, final) == int(final == 0 and n > 8192)
+
+
+def test_f16_workspace_and_shape_errors(L):
+    # q' [B][T][H][64] fp16 plus V^T [B][H][64][round_up(N, 128)] fp16
+    w = binding.workspace_size(binding.OP_ICL_ATTENTION_F16, 2, 1000, 24, 3)
+    assert w >= 256 + 2 * 1024 * 3 * 64 * 2 + 2 * 3 * 64 * 1024 * 2
+    assert binding.workspace_size(binding.OP_ICL_ATTENTION_F16, 1, 0, 8, 4) == 0
+    assert L.sdm_icl_attention_f16(None, None, None, 1, 0, 5, 4, 64, None, None, None, None, 0, None) == 1
+    assert L.sdm_icl_attention_f16(None, None, None, 1, 10, 5, 4, 48, None, None, None, None, 0, None) == 2
+    assert L.sdm_icl_attention_f16(None, None, None, 1, 10, 5, 200, 64, None, None, None, None, 0, None) == 2
