@@ -385,15 +385,34 @@ def run_per_kernel(args):
          # all of them again and writes e4m3 (3 B): both passes are inherent
          2 * 3 * el(N) + 3 * (el(T) + 2 * el(N)), 0.0),
         ("a3 FP8 attention (sdm_fp8_attention)", lambda: sdm.fp8_attention(q8, cache, out=out, ws=ws_a),
-         el(T) + 2 * el(N) + 2 * el(T), attn_flops(T, N, H)),
+         el(T) + 2 * el(N) + 2 * el(T), B * attn_flops(T, N, H)),
         ("a4 cached prediction, 1024 queries (sdm_cached_attention)",
          lambda: sdm.cached_attention(queries, cache, c_h, gate=None, out=pred, ws=ws_c),
-         2 * el(Mq) + 2 * el(N) + 2 * el(Mq), attn_flops(Mq, N, H)),
+         2 * el(Mq) + 2 * el(N) + 2 * el(Mq), B * attn_flops(Mq, N, H)),
         ("a5 fp16 attention, query scaling included (sdm_icl_attention_f16)",
          lambda: sdm.icl_attention_f16(q, k, v, N, c_h, gate, out=out, ws=ws_h),
          # q -> q' (4 B), V -> V^T (4 B), then q', K, V^T read and O written (2 B each)
-         4 * el(T) + 4 * el(N) + 2 * el(T) + 4 * el(N) + 2 * el(T), attn_flops(T, N, H)),
+         4 * el(T) + 4 * el(N) + 2 * el(T) + 4 * el(N) + 2 * el(T), B * attn_flops(T, N, H)),
     ]
+    lens = inp.get("ctx_len")
+    if lens is not None:
+        # batched estimators with padded contexts: only the unmasked rows are work
+        useful = sum(attn_flops(int(n) + M, int(n), H) for n in lens)
+        ctx = sum(int(n) for n in lens) * H * 64          # unmasked context elements
+        rows = sum(int(n) + M for n in lens) * H * 64     # elements of the rows that attend
+        cache_r = sdm.FP8Cache(B, N, H, device)
+        ws_r = sdm.new_workspace(sdm.workspace_size(binding.OP_ICL_ATTENTION, B, N, M, H), device)
+        steps += [
+            ("a6 ragged batch, FP8 one-call layer (sdm_icl_attention_ragged)",
+             lambda: sdm.icl_attention(q, k, v, N, c_h, gate, cache=cache_r, out=out, ws=ws_r, ctx_len=lens),
+             # amax reads Q', K, V context rows (2 B); quantisation reads them again and the query
+             # rows and writes e4m3 (3 B); attention reads the e4m3 tensors and writes O (2 B)
+             6 * ctx + (3 * rows + 6 * ctx) + (rows + 2 * ctx) + 2 * rows, useful),
+            ("a7 ragged batch, fp16 attention (sdm_icl_attention_f16_ragged)",
+             lambda: sdm.icl_attention_f16(q, k, v, N, c_h, gate, out=out, ws=ws_h, ctx_len=lens),
+             # q -> q' (4 B), V -> V^T (4 B), then q', K, V^T read and O written (2 B each)
+             4 * rows + 4 * ctx + 2 * rows + 4 * ctx + 2 * rows, useful),
+        ]
     # a filled cache and Q8 for the attention steps
     q8.copy_(sdm.fp8_quantize_context(sdm.qscale_fused(q, c_h, N, gate), k, v, N, cache=cache)[0])
     for name, fn, nbytes, flops in steps:
@@ -411,8 +430,8 @@ def run_per_kernel(args):
                 "gbs": nbytes / (ms * 1e-3) / 1e9, "frac_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm}
         if flops:
             tf = flops / (ms * 1e-3) / 1e12
-            line.update({"tflops": tf, "frac_f16" if name.startswith("a5") else "frac_fp8":
-                         tf / (f16 if name.startswith("a5") else fp8)})
+            is_f16 = name.startswith("a5") or name.startswith("a7")
+            line.update({"tflops": tf, "frac_f16" if is_f16 else "frac_fp8": tf / (f16 if is_f16 else fp8)})
         print(json.dumps(line), flush=True)
 
 

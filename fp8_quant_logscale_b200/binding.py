@@ -26,8 +26,8 @@ HEAD_DIM = 64
 # Every symbol the header declares (checked by the ABI tests).
 EXPORTS = ("sdm_status_string", "sdm_version", "sdm_split_keys", "sdm_cache_layout", "sdm_workspace_size", "sdm_qscale_fused",
            "sdm_fp8_quantize_context", "sdm_fp8_quantize_context_noalloc", "sdm_fp8_attention", "sdm_icl_attention",
-           "sdm_cached_attention", "sdm_fp8_eligible", "sdm_icl_attention_f16", "sdm_sync_status",
-           "sdm_selftest_wait_timeout")
+           "sdm_cached_attention", "sdm_fp8_eligible", "sdm_icl_attention_f16", "sdm_icl_attention_ragged",
+           "sdm_icl_attention_f16_ragged", "sdm_sync_status", "sdm_selftest_wait_timeout")
 NOALLOC_MAX_BATCH_HEADS = 4096
 
 
@@ -41,7 +41,7 @@ class CacheStruct(ctypes.Structure):
     _fields_ = [("k8", ctypes.c_void_p), ("v8t", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("n_ctx", ctypes.c_int64), ("ld_v", ctypes.c_int64), ("batch", ctypes.c_int32),
                 ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("device", ctypes.c_int32),
-                ("filled", ctypes.c_int32)]
+                ("filled", ctypes.c_int32), ("ragged", ctypes.c_int32)]
 
 
 _lib = None
@@ -83,6 +83,12 @@ def lib() -> ctypes.CDLL:
         L.sdm_cached_attention.restype = ctypes.c_int
         L.sdm_cached_attention.argtypes = [_P, _I32, _I64, _I32, _I32, ctypes.POINTER(CacheStruct), _P, _P, _P,
                                            _P, _SZ, _P]
+        L.sdm_icl_attention_ragged.restype = ctypes.c_int
+        L.sdm_icl_attention_ragged.argtypes = [_P, _P, _P, _I32, _I64, _I64, _I32, _I32, _P, _P, _P, _P,
+                                               ctypes.POINTER(CacheStruct), _P, _SZ, _P]
+        L.sdm_icl_attention_f16_ragged.restype = ctypes.c_int
+        L.sdm_icl_attention_f16_ragged.argtypes = [_P, _P, _P, _I32, _I64, _I64, _I32, _I32, _P, _P, _P, _P,
+                                                   _P, _SZ, _P]
         L.sdm_fp8_eligible.restype = _I32
         L.sdm_fp8_eligible.argtypes = [_I64, _I32]
         L.sdm_icl_attention_f16.restype = ctypes.c_int
@@ -154,8 +160,17 @@ def selftest_wait_timeout(ws: torch.Tensor, limit_cycles: int = 1_000_000) -> No
                "sdm_selftest_wait_timeout")
 
 
+def _ctx_len_array(ctx_len, batch: int):
+    """Host int64 array of the per-batch context lengths (ragged batches)."""
+    lens = [int(x) for x in ctx_len]
+    if len(lens) != batch:
+        raise ValueError(f"ctx_len has {len(lens)} entries for batch {batch}")
+    return (ctypes.c_int64 * batch)(*lens)
+
+
 class FP8Cache:
-    """Caller-owned FP8 K/V cache (k8 [B,H,N,64], v8t [B,H,64,ld_v], scales [3,B,H])."""
+    """Caller-owned FP8 K/V cache (k8 [B,H,N,64], v8t [B,H,64,ld_v], scales block: scales [3,B,H]
+    followed by the per-batch context lengths of a ragged fit)."""
 
     def __init__(self, batch: int, n_ctx: int, heads: int, device):
         kb, vb, sb, ld = _SZ(), _SZ(), _SZ(), _I64()
@@ -166,10 +181,23 @@ class FP8Cache:
             device = torch.device("cuda", torch.cuda.current_device())
         self.k8 = torch.empty((batch, heads, n_ctx, HEAD_DIM), dtype=torch.uint8, device=device)
         self.v8t = torch.empty((batch, heads, HEAD_DIM, ld.value), dtype=torch.uint8, device=device)
-        self.scales = torch.empty((3, batch, heads), dtype=torch.float32, device=device)
-        assert self.k8.numel() == kb.value and self.v8t.numel() == vb.value and self.scales.numel() * 4 == sb.value
-        self.struct = CacheStruct(self.k8.data_ptr(), self.v8t.data_ptr(), self.scales.data_ptr(), n_ctx, ld.value,
-                                  batch, heads, HEAD_DIM, device.index, 0)
+        self.block = torch.zeros(sb.value // 4, dtype=torch.float32, device=device)
+        self.scales = self.block[:3 * batch * heads].view(3, batch, heads)
+        assert self.k8.numel() == kb.value and self.v8t.numel() == vb.value and self.block.numel() * 4 == sb.value
+        self.struct = CacheStruct(self.k8.data_ptr(), self.v8t.data_ptr(), self.block.data_ptr(), n_ctx, ld.value,
+                                  batch, heads, HEAD_DIM, device.index, 0, 0)
+        self.batch, self.heads = batch, heads
+
+    @property
+    def ragged(self) -> bool:
+        return self.struct.ragged == 1
+
+    def ctx_len(self) -> list[int]:
+        """Per-batch context lengths (n_ctx for every batch unless the fit was ragged)."""
+        if not self.ragged:
+            return [self.n_ctx] * self.batch
+        off = 3 * self.batch * self.heads
+        return self.block[off:off + self.batch].view(torch.int32).tolist()
 
     @property
     def filled(self) -> bool:
@@ -257,8 +285,11 @@ def fp8_attention(q8: torch.Tensor, cache: FP8Cache, split: bool = False, out: t
 
 def icl_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_ctx: int, c_h: torch.Tensor,
                   gate: torch.Tensor | None = None, cache: FP8Cache | None = None, out: torch.Tensor | None = None,
-                  ws: torch.Tensor | None = None) -> torch.Tensor:
-    """One call of the layer: q [B,T,H,64] raw fp16, k/v [B,N,H,64] fp16 -> out [B,T,H,64] fp16."""
+                  ws: torch.Tensor | None = None, ctx_len=None) -> torch.Tensor:
+    """One call of the layer: q [B,T,H,64] raw fp16, k/v [B,N,H,64] fp16 -> out [B,T,H,64] fp16.
+
+    ctx_len (B ints, 1 <= n_b <= n_ctx): ragged batch; rows [n_b, n_ctx) of batch b are padding.
+    """
     _want(q, torch.float16, "q", 4)
     _want(k, torch.float16, "k", 4)
     _want(v, torch.float16, "v", 4)
@@ -271,10 +302,15 @@ def icl_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_ctx: int,
     out = torch.empty_like(q) if out is None else out
     need = workspace_size(OP_ICL_ATTENTION, B, n_ctx, M, H, keep_cache=cache is not None)
     ws = new_workspace(need, dev) if ws is None else ws
+    cs = None if cache is None else ctypes.byref(cache.struct)
     with torch.cuda.device(dev):
-        _check(lib().sdm_icl_attention(_ptr(q), _ptr(k), _ptr(v), B, n_ctx, M, H, d, _ptr(c_h), _ptr(gate),
-                                       _ptr(out), None if cache is None else ctypes.byref(cache.struct), _ptr(ws),
-                                       ws.numel(), _stream(dev)), "sdm_icl_attention")
+        if ctx_len is None:
+            _check(lib().sdm_icl_attention(_ptr(q), _ptr(k), _ptr(v), B, n_ctx, M, H, d, _ptr(c_h), _ptr(gate),
+                                           _ptr(out), cs, _ptr(ws), ws.numel(), _stream(dev)), "sdm_icl_attention")
+        else:
+            _check(lib().sdm_icl_attention_ragged(_ptr(q), _ptr(k), _ptr(v), B, n_ctx, M, H, d,
+                                                  _ctx_len_array(ctx_len, B), _ptr(c_h), _ptr(gate), _ptr(out), cs,
+                                                  _ptr(ws), ws.numel(), _stream(dev)), "sdm_icl_attention_ragged")
     return out
 
 
@@ -303,10 +339,11 @@ def fp8_eligible(n_unmasked_ctx: int, final_layer: bool = False) -> bool:
 
 def icl_attention_f16(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_ctx: int, c_h: torch.Tensor | None,
                       gate: torch.Tensor | None = None, out: torch.Tensor | None = None,
-                      ws: torch.Tensor | None = None) -> torch.Tensor:
+                      ws: torch.Tensor | None = None, ctx_len=None) -> torch.Tensor:
     """Normal-precision layer call: q [B,T,H,64] raw fp16, k/v [B,N,H,64] fp16 -> out [B,T,H,64] fp16.
 
-    c_h None: no query scaling (q is used as given; gate must be None).
+    c_h None: no query scaling (q is used as given; gate must be None).  ctx_len: ragged batch
+    as for icl_attention.
     """
     _want(q, torch.float16, "q", 4)
     _want(k, torch.float16, "k", 4)
@@ -322,20 +359,29 @@ def icl_attention_f16(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_ctx: 
     need = workspace_size(OP_ICL_ATTENTION_F16, B, n_ctx, M, H)
     ws = new_workspace(need, dev) if ws is None else ws
     with torch.cuda.device(dev):
-        _check(lib().sdm_icl_attention_f16(_ptr(q), _ptr(k), _ptr(v), B, n_ctx, M, H, d, _ptr(c_h), _ptr(gate),
-                                           _ptr(out), _ptr(ws), ws.numel(), _stream(dev)), "sdm_icl_attention_f16")
+        if ctx_len is None:
+            _check(lib().sdm_icl_attention_f16(_ptr(q), _ptr(k), _ptr(v), B, n_ctx, M, H, d, _ptr(c_h),
+                                               _ptr(gate), _ptr(out), _ptr(ws), ws.numel(), _stream(dev)),
+                   "sdm_icl_attention_f16")
+        else:
+            _check(lib().sdm_icl_attention_f16_ragged(_ptr(q), _ptr(k), _ptr(v), B, n_ctx, M, H, d,
+                                                      _ctx_len_array(ctx_len, B), _ptr(c_h), _ptr(gate), _ptr(out),
+                                                      _ptr(ws), ws.numel(), _stream(dev)),
+                   "sdm_icl_attention_f16_ragged")
     return out
 
 
 def icl_layer(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_ctx: int, c_h: torch.Tensor,
               gate: torch.Tensor | None = None, final_layer: bool = False, cache: FP8Cache | None = None,
-              out: torch.Tensor | None = None) -> torch.Tensor:
+              out: torch.Tensor | None = None, ctx_len=None) -> torch.Tensor:
     """One ICL attention layer with the precision rule applied: FP8 (icl_attention) when
-    fp8_eligible(n_ctx, final_layer), else normal precision (icl_attention_f16).  A cache
-    can only be filled on the FP8 path."""
-    if fp8_eligible(n_ctx, final_layer):
-        return icl_attention(q, k, v, n_ctx, c_h, gate=gate, cache=cache, out=out)
+    fp8_eligible(n, final_layer), else normal precision (icl_attention_f16).  n is the number of
+    unmasked context rows: n_ctx, or for a ragged batch the smallest n_b (FP8 only when every
+    estimator of the batch qualifies).  A cache can only be filled on the FP8 path."""
+    n_unmasked = n_ctx if ctx_len is None else min(int(x) for x in ctx_len)
+    if fp8_eligible(n_unmasked, final_layer):
+        return icl_attention(q, k, v, n_ctx, c_h, gate=gate, cache=cache, out=out, ctx_len=ctx_len)
     if cache is not None:
         raise ValueError("an FP8 cache is filled only by an FP8-eligible layer "
-                         f"(n_ctx={n_ctx}, final_layer={final_layer})")
-    return icl_attention_f16(q, k, v, n_ctx, c_h, gate=gate, out=out)
+                         f"(unmasked context rows={n_unmasked}, final_layer={final_layer})")
+    return icl_attention_f16(q, k, v, n_ctx, c_h, gate=gate, out=out, ctx_len=ctx_len)

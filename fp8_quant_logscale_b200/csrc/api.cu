@@ -77,7 +77,7 @@ sdm_status check_tensor(const void* p, int dev) {
 // Workspace carve-up.  Offsets are 1 KB aligned; the error word sits at 0.
 struct WsLayout {
   size_t amax = 0, gate_w = 0, q8 = 0, k8 = 0, v8t = 0, scales = 0, part_acc = 0, part_ml = 0, total = 0;
-  size_t q16 = 0, vt16 = 0;  // normal-precision path: q' and V^T in fp16
+  size_t q16 = 0, vt16 = 0, meta = 0;  // normal-precision path: q', V^T in fp16, ragged meta
 };
 
 int64_t n_splits_for(int64_t n_ctx) {
@@ -95,6 +95,8 @@ WsLayout ws_layout(sdm_op op, int32_t B, int64_t N, int64_t M, int32_t H, int32_
     off = align_up(off + BH * (size_t)(N + M) * kHeadDim * sizeof(uint16_t), kAlign);
     w.vt16 = off;
     off = align_up(off + BH * kHeadDim * (size_t)ld * sizeof(uint16_t), kAlign);
+    w.meta = off;  // ragged contexts: n_b int32 [B], lam_b fp32 [B]
+    off = align_up(off + 2 * (size_t)B * sizeof(float), kAlign);
     w.total = off;
     return w;
   }
@@ -115,8 +117,8 @@ WsLayout ws_layout(sdm_op op, int32_t B, int64_t N, int64_t M, int32_t H, int32_
     off = align_up(off + BH * (size_t)N * kHeadDim, kAlign);
     w.v8t = off;
     off = align_up(off + BH * kHeadDim * (size_t)ld, kAlign);
-    w.scales = off;
-    off = align_up(off + 3 * BH * sizeof(float), kAlign);
+    w.scales = off;  // scales block: [3][B][H] scales, then the ragged meta words
+    off = align_up(off + scales_block_words(B, H, true) * sizeof(float), kAlign);
   }
   if (op == SDM_OP_CACHED_ATTENTION) {
     const size_t S = (size_t)n_splits_for(N);
@@ -140,7 +142,7 @@ sdm_status check_ws(void* ws, size_t ws_bytes, size_t need, int dev) {
 sdm_status check_cache(const sdm_fp8_cache* c, int32_t B, int32_t H, int32_t d, int dev, bool need_filled) {
   if (c == nullptr) return SDM_ERR_INVALID_ARG;
   if (c->batch != B || c->heads != H || c->head_dim != d || c->device != dev || c->n_ctx < 1 ||
-      c->ld_v != round_up(c->n_ctx, kKvTile))
+      c->ld_v != round_up(c->n_ctx, kKvTile) || (c->ragged != 0 && c->ragged != 1))
     return SDM_ERR_CACHE_MISMATCH;
   if (need_filled && c->filled != 1) return SDM_ERR_CACHE_MISMATCH;
   if (c->k8 == nullptr || c->v8t == nullptr || c->scales == nullptr) return SDM_ERR_INVALID_ARG;
@@ -158,6 +160,7 @@ QScale make_qscale(int64_t n_len, const float* c_h, const void* gate) {
   qs.c_h = c_h;
   qs.gate = reinterpret_cast<const __half*>(gate);
   qs.gate_w = nullptr;
+  qs.lam_b = nullptr;
   return qs;
 }
 
@@ -168,6 +171,7 @@ QScale no_qscale() {
   qs.c_h = nullptr;
   qs.gate = nullptr;
   qs.gate_w = nullptr;
+  qs.lam_b = nullptr;
   return qs;
 }
 
@@ -181,21 +185,56 @@ cudaError_t prepare_gate(QScale& qs, int64_t n, uint8_t* ws_base, const WsLayout
   return e;
 }
 
+// Ragged contexts: checks the host array ctx_len[B] (1 <= n_b <= N) and
+// enqueues the writes of n_b and lam_b = fp32 ln(n_b) (the host evaluation the
+// uniform path uses) into the meta words at `meta` (n_b int32 [B], lam_b fp32 [B]).
+sdm_status check_ctx_len(const int64_t* ctx_len, int32_t B, int64_t N) {
+  if (ctx_len == nullptr) return SDM_ERR_INVALID_ARG;
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, ctx_len) == cudaSuccess) {
+    if (at.type == cudaMemoryTypeDevice) return SDM_ERR_INVALID_ARG;  // must be host memory
+  } else {
+    cudaGetLastError();
+  }
+  for (int32_t b = 0; b < B; ++b)
+    if (ctx_len[b] < 1 || ctx_len[b] > N) return SDM_ERR_INVALID_ARG;
+  return SDM_OK;
+}
+
+cudaError_t put_meta(const int64_t* ctx_len, int32_t B, float* meta, cudaStream_t st) {
+  int32_t* n_dst = reinterpret_cast<int32_t*>(meta);
+  float* lam_dst = meta + B;
+  for (int32_t b0 = 0; b0 < B; b0 += kMetaChunk) {
+    MetaChunk c;
+    memset(&c, 0, sizeof(c));
+    c.b0 = b0;
+    c.count = B - b0 < kMetaChunk ? B - b0 : kMetaChunk;
+    for (int i = 0; i < c.count; ++i) {
+      c.n[i] = static_cast<int32_t>(ctx_len[b0 + i]);
+      c.lam[i] = logf(static_cast<float>(ctx_len[b0 + i]));
+    }
+    const cudaError_t e = launch_write_meta(c, n_dst, lam_dst, st);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 // amax -> scales -> Q8 / K8 / V8^T.  `qs` is applied to Q (enabled: raw q in).
+// n_valid (device, nullable): per-batch context rows; padding rows get zero codes.
 sdm_status run_quantize(const __half* q, const __half* k, const __half* v, int32_t B, int64_t N, int64_t M,
                         int32_t H, QScale qs, uint8_t* q8, uint8_t* k8, uint8_t* v8t, int64_t ld, float* scales,
-                        uint8_t* ws_base, const WsLayout& w, cudaStream_t st) {
+                        const int32_t* n_valid, uint8_t* ws_base, const WsLayout& w, cudaStream_t st) {
   const int64_t T = N + M;
   uint32_t* amax = reinterpret_cast<uint32_t*>(ws_base + w.amax);
   SDM_CUDA(cudaMemsetAsync(amax, 0, 3 * (size_t)B * H * sizeof(uint32_t), st));
   SDM_CUDA(prepare_gate(qs, (int64_t)B * T * H, ws_base, w, st));
   RowsDesc dq{q, B, H, T}, dk{k, B, H, N}, dv{v, B, H, N};
-  SDM_CUDA(launch_context_amax(dq, qs, dk, dv, N, amax, st));
+  SDM_CUDA(launch_context_amax(dq, qs, dk, dv, N, n_valid, amax, st));
   SDM_CUDA(launch_scales_from_amax(amax, B * H, scales, st));
   const int64_t BH = (int64_t)B * H;
-  SDM_CUDA(launch_quantize_rows(dq, qs, T, scales, q8, T, st));
-  SDM_CUDA(launch_quantize_rows(dk, no_qscale(), N, scales + BH, k8, N, st));
-  SDM_CUDA(launch_quantize_vt(dv, N, scales + 2 * BH, v8t, ld, st));
+  SDM_CUDA(launch_quantize_rows(dq, qs, T, scales, q8, T, n_valid, N, st));
+  SDM_CUDA(launch_quantize_rows(dk, no_qscale(), N, scales + BH, k8, N, n_valid, N, st));
+  SDM_CUDA(launch_quantize_vt(dv, N, n_valid, scales + 2 * BH, v8t, ld, st));
   return SDM_OK;
 }
 
@@ -217,7 +256,7 @@ const char* sdm_status_string(sdm_status s) {
   return "SDM_ERR_UNKNOWN";
 }
 
-int32_t sdm_version(void) { return 100; }
+int32_t sdm_version(void) { return 101; }
 
 int64_t sdm_split_keys(int64_t n_ctx) { return n_ctx < 1 ? 0 : split_keys_for(n_ctx); }
 
@@ -228,7 +267,7 @@ sdm_status sdm_cache_layout(int32_t B, int64_t N, int32_t H, int32_t d, size_t* 
   const int64_t ld = round_up(N, kKvTile);
   if (k8_bytes) *k8_bytes = (size_t)B * H * N * kHeadDim;
   if (v8t_bytes) *v8t_bytes = (size_t)B * H * kHeadDim * ld;
-  if (scales_bytes) *scales_bytes = 3 * (size_t)B * H * sizeof(float);
+  if (scales_bytes) *scales_bytes = scales_block_words(B, H, true) * sizeof(float);
   if (ld_v) *ld_v = ld;
   return SDM_OK;
 }
@@ -279,8 +318,9 @@ sdm_status sdm_fp8_quantize_context(const void* q_scaled, const void* k, const v
   cudaStream_t st = as_stream(stream);
   SDM_TRY(run_quantize(reinterpret_cast<const __half*>(q_scaled), reinterpret_cast<const __half*>(k),
                        reinterpret_cast<const __half*>(v), B, N, M, H, no_qscale(), q8, cache->k8, cache->v8t,
-                       cache->ld_v, cache->scales, reinterpret_cast<uint8_t*>(ws), w, st));
+                       cache->ld_v, cache->scales, nullptr, reinterpret_cast<uint8_t*>(ws), w, st));
   cache->filled = 1;
+  cache->ragged = 0;
   return SDM_OK;
 }
 
@@ -314,16 +354,20 @@ sdm_status sdm_fp8_attention(const uint8_t* q8, int32_t B, int64_t rows, const s
   a.part_acc = split ? reinterpret_cast<float*>(base + w.part_acc) : nullptr;
   a.part_ml = split ? reinterpret_cast<float*>(base + w.part_ml) : nullptr;
   a.err = reinterpret_cast<uint32_t*>(base);
+  a.n_keys = cache->ragged ? reinterpret_cast<const int32_t*>(cache->scales + 3 * (int64_t)B * H) : nullptr;
+  a.pad_rows = false;
   SDM_CUDA(launch_attention(q8, cache->k8, cache->v8t, a, st));
   if (split) SDM_CUDA(launch_splitkv_reduce(a, st));
   return SDM_OK;
 }
 
-sdm_status sdm_icl_attention(const void* q, const void* k, const void* v, int32_t B, int64_t N, int64_t M,
-                             int32_t H, int32_t d, const float* c_h, const void* gate, void* out,
-                             sdm_fp8_cache* cache, void* ws, size_t ws_bytes, void* stream) {
+static sdm_status icl_attention_impl(const void* q, const void* k, const void* v, int32_t B, int64_t N, int64_t M,
+                                     int32_t H, int32_t d, const int64_t* ctx_len, const float* c_h,
+                                     const void* gate, void* out, sdm_fp8_cache* cache, void* ws, size_t ws_bytes,
+                                     void* stream) {
   SDM_TRY(check_shape(B, N, M, H, d));
   if (N < 1) return SDM_ERR_INVALID_ARG;
+  if (ctx_len != nullptr) SDM_TRY(check_ctx_len(ctx_len, B, N));
   const int dev = current_device();
   if (dev < 0) return SDM_ERR_CUDA;
   SDM_TRY(check_tensor(q, dev));
@@ -357,13 +401,23 @@ sdm_status sdm_icl_attention(const void* q, const void* k, const void* v, int32_
     local.heads = H;
     local.head_dim = d;
     local.device = dev;
+    local.ragged = 0;
     c = &local;
   }
   uint8_t* q8 = base + w.q8;
+  QScale qs = make_qscale(N, c_h, gate);
+  const int32_t* n_valid = nullptr;
+  if (ctx_len != nullptr) {
+    float* meta = c->scales + 3 * (int64_t)B * H;
+    SDM_CUDA(put_meta(ctx_len, B, meta, st));
+    n_valid = reinterpret_cast<const int32_t*>(meta);
+    qs.lam_b = meta + B;
+  }
   SDM_TRY(run_quantize(reinterpret_cast<const __half*>(q), reinterpret_cast<const __half*>(k),
-                       reinterpret_cast<const __half*>(v), B, N, M, H, make_qscale(N, c_h, gate), q8, c->k8, c->v8t,
-                       c->ld_v, c->scales, base, w, st));
+                       reinterpret_cast<const __half*>(v), B, N, M, H, qs, q8, c->k8, c->v8t, c->ld_v, c->scales,
+                       n_valid, base, w, st));
   c->filled = 1;
+  c->ragged = ctx_len != nullptr ? 1 : 0;
   AttnArgs a;
   a.B = B;
   a.H = H;
@@ -378,9 +432,27 @@ sdm_status sdm_icl_attention(const void* q, const void* k, const void* v, int32_
   a.part_acc = nullptr;
   a.part_ml = nullptr;
   a.err = reinterpret_cast<uint32_t*>(base);
+  a.n_keys = n_valid;
+  a.pad_rows = n_valid != nullptr;
   SDM_CUDA(launch_attention(q8, c->k8, c->v8t, a, st));
   return SDM_OK;
 }
+
+sdm_status sdm_icl_attention(const void* q, const void* k, const void* v, int32_t B, int64_t N, int64_t M,
+                             int32_t H, int32_t d, const float* c_h, const void* gate, void* out,
+                             sdm_fp8_cache* cache, void* ws, size_t ws_bytes, void* stream) {
+  return icl_attention_impl(q, k, v, B, N, M, H, d, nullptr, c_h, gate, out, cache, ws, ws_bytes, stream);
+}
+
+sdm_status sdm_icl_attention_ragged(const void* q, const void* k, const void* v, int32_t B, int64_t N, int64_t M,
+                                    int32_t H, int32_t d, const int64_t* ctx_len, const float* c_h,
+                                    const void* gate, void* out, sdm_fp8_cache* cache, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  if (ctx_len == nullptr) return SDM_ERR_INVALID_ARG;
+  return icl_attention_impl(q, k, v, B, N, M, H, d, ctx_len, c_h, gate, out, cache, ws, ws_bytes, stream);
+}
+
+
 
 sdm_status sdm_cached_attention(const void* q, int32_t B, int64_t M, int32_t H, int32_t d,
                                 const sdm_fp8_cache* cache, const float* c_h, const void* gate, void* out, void* ws,
@@ -406,10 +478,13 @@ sdm_status sdm_cached_attention(const void* q, int32_t B, int64_t M, int32_t H, 
   uint8_t* base = reinterpret_cast<uint8_t*>(ws);
   uint8_t* q8 = base + w.q8;
   // query scaling with the shared key length n = N, quantised with the context s_q
+  // (ragged cache: with the batch's own n_b and keys [0, n_b))
   RowsDesc dq{reinterpret_cast<const __half*>(q), B, H, M};
   QScale qs = make_qscale(N, c_h, gate);
+  const float* meta = cache->scales + 3 * (int64_t)B * H;
+  if (cache->ragged) qs.lam_b = meta + B;
   SDM_CUDA(prepare_gate(qs, (int64_t)B * M * H, base, w, st));
-  SDM_CUDA(launch_quantize_rows(dq, qs, M, cache->scales, q8, M, st));
+  SDM_CUDA(launch_quantize_rows(dq, qs, M, cache->scales, q8, M, nullptr, 0, st));
   AttnArgs a;
   a.B = B;
   a.H = H;
@@ -424,6 +499,8 @@ sdm_status sdm_cached_attention(const void* q, int32_t B, int64_t M, int32_t H, 
   a.part_acc = reinterpret_cast<float*>(base + w.part_acc);
   a.part_ml = reinterpret_cast<float*>(base + w.part_ml);
   a.err = reinterpret_cast<uint32_t*>(base);
+  a.n_keys = cache->ragged ? reinterpret_cast<const int32_t*>(meta) : nullptr;
+  a.pad_rows = false;
   SDM_CUDA(launch_attention(q8, cache->k8, cache->v8t, a, st));
   SDM_CUDA(launch_splitkv_reduce(a, st));
   return SDM_OK;
@@ -433,11 +510,12 @@ int32_t sdm_fp8_eligible(int64_t n_unmasked_ctx, int32_t final_layer) {
   return (final_layer == 0 && n_unmasked_ctx > SDM_FP8_MIN_CONTEXT) ? 1 : 0;
 }
 
-sdm_status sdm_icl_attention_f16(const void* q, const void* k, const void* v, int32_t B, int64_t N, int64_t M,
-                                 int32_t H, int32_t d, const float* c_h, const void* gate, void* out, void* ws,
-                                 size_t ws_bytes, void* stream) {
+static sdm_status icl_attention_f16_impl(const void* q, const void* k, const void* v, int32_t B, int64_t N,
+                                         int64_t M, int32_t H, int32_t d, const int64_t* ctx_len, const float* c_h,
+                                         const void* gate, void* out, void* ws, size_t ws_bytes, void* stream) {
   SDM_TRY(check_shape(B, N, M, H, d));
   if (N < 1) return SDM_ERR_INVALID_ARG;
+  if (ctx_len != nullptr) SDM_TRY(check_ctx_len(ctx_len, B, N));
   const int dev = current_device();
   if (dev < 0) return SDM_ERR_CUDA;
   SDM_TRY(check_tensor(q, dev));
@@ -458,19 +536,44 @@ sdm_status sdm_icl_attention_f16(const void* q, const void* k, const void* v, in
   uint8_t* base = reinterpret_cast<uint8_t*>(ws);
   const int64_t T = N + M;
   const int64_t ld = round_up(N, kKvTile);
+  const int32_t* n_valid = nullptr;
+  const float* lam_b = nullptr;
+  if (ctx_len != nullptr) {
+    float* meta = reinterpret_cast<float*>(base + w.meta);
+    SDM_CUDA(put_meta(ctx_len, B, meta, st));
+    n_valid = reinterpret_cast<const int32_t*>(meta);
+    lam_b = meta + B;
+  }
   const __half* qs = reinterpret_cast<const __half*>(q);
   if (c_h != nullptr) {
     __half* q16 = reinterpret_cast<__half*>(base + w.q16);
-    SDM_CUDA(launch_qscale(qs, q16, B, T, H, make_qscale(N, c_h, gate), st));
+    QScale sc = make_qscale(N, c_h, gate);
+    sc.lam_b = lam_b;
+    SDM_CUDA(launch_qscale(qs, q16, B, T, H, sc, st));
     qs = q16;
   }
   __half* vt16 = reinterpret_cast<__half*>(base + w.vt16);
   RowsDesc dv{reinterpret_cast<const __half*>(v), B, H, N};
-  SDM_CUDA(launch_transpose_vt_f16(dv, N, vt16, ld, st));
-  SDM_CUDA(launch_attention_f16(qs, reinterpret_cast<const __half*>(k), vt16, B, T, N, H, ld,
+  SDM_CUDA(launch_transpose_vt_f16(dv, N, n_valid, vt16, ld, st));
+  SDM_CUDA(launch_attention_f16(qs, reinterpret_cast<const __half*>(k), vt16, B, T, N, H, ld, n_valid,
                                 reinterpret_cast<__half*>(out), reinterpret_cast<uint32_t*>(base), st));
   return SDM_OK;
 }
+
+sdm_status sdm_icl_attention_f16(const void* q, const void* k, const void* v, int32_t B, int64_t N, int64_t M,
+                                 int32_t H, int32_t d, const float* c_h, const void* gate, void* out, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  return icl_attention_f16_impl(q, k, v, B, N, M, H, d, nullptr, c_h, gate, out, ws, ws_bytes, stream);
+}
+
+sdm_status sdm_icl_attention_f16_ragged(const void* q, const void* k, const void* v, int32_t B, int64_t N,
+                                        int64_t M, int32_t H, int32_t d, const int64_t* ctx_len, const float* c_h,
+                                        const void* gate, void* out, void* ws, size_t ws_bytes, void* stream) {
+  if (ctx_len == nullptr) return SDM_ERR_INVALID_ARG;
+  return icl_attention_f16_impl(q, k, v, B, N, M, H, d, ctx_len, c_h, gate, out, ws, ws_bytes, stream);
+}
+
+
 
 sdm_status sdm_selftest_wait_timeout(void* ws, int64_t limit_cycles, void* stream) {
   if (ws == nullptr || !aligned(ws, 256)) return SDM_ERR_INVALID_ARG;
@@ -569,11 +672,12 @@ extern "C" sdm_status sdm_fp8_quantize_context_noalloc(const void* q_scaled, con
   RowsDesc dq{reinterpret_cast<const __half*>(q_scaled), B, H, T};
   RowsDesc dk{reinterpret_cast<const __half*>(k), B, H, N};
   RowsDesc dv{reinterpret_cast<const __half*>(v), B, H, N};
-  SDM_CUDA(launch_context_amax(dq, no_qscale(), dk, dv, N, amax, st));
+  SDM_CUDA(launch_context_amax(dq, no_qscale(), dk, dv, N, nullptr, amax, st));
   SDM_CUDA(launch_scales_from_amax(amax, B * H, cache->scales, st));
-  SDM_CUDA(launch_quantize_rows(dq, no_qscale(), T, cache->scales, q8, T, st));
-  SDM_CUDA(launch_quantize_rows(dk, no_qscale(), N, cache->scales + BH, cache->k8, N, st));
-  SDM_CUDA(launch_quantize_vt(dv, N, cache->scales + 2 * BH, cache->v8t, cache->ld_v, st));
+  SDM_CUDA(launch_quantize_rows(dq, no_qscale(), T, cache->scales, q8, T, nullptr, 0, st));
+  SDM_CUDA(launch_quantize_rows(dk, no_qscale(), N, cache->scales + BH, cache->k8, N, nullptr, 0, st));
+  SDM_CUDA(launch_quantize_vt(dv, N, nullptr, cache->scales + 2 * BH, cache->v8t, cache->ld_v, st));
   cache->filled = 1;
+  cache->ragged = 0;
   return SDM_OK;
 }

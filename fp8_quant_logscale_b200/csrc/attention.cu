@@ -96,6 +96,8 @@ struct KParams {
   float* part_acc;
   float* part_ml;
   uint32_t* err;
+  const int32_t* n_keys;  // [B] keys per batch, or nullptr: N
+  int32_t pad_rows;       // rows [n_b, N) are padding: written as zeros
 };
 
 template <class S>
@@ -173,9 +175,13 @@ __global__ void __launch_bounds__(Cfg<kTiles>::kThreads, Cfg<kTiles>::kMinBlocks
   const int64_t split = rest % p.n_splits;
   const int64_t bh = rest / p.n_splits;
   const int64_t row0 = pair * (kTiles * kQTile);
+  const int64_t n_b = p.n_keys != nullptr ? (int64_t)__ldg(p.n_keys + bh / p.H) : p.N;  // this batch's keys
   const int64_t kv_begin = p.partial ? split * p.split_keys : 0;
-  const int64_t kv_end = p.partial ? min(p.N, kv_begin + p.split_keys) : p.N;
-  const int n_tiles = static_cast<int>((kv_end - kv_begin + kKvTile - 1) / kKvTile);
+  const int64_t kv_end = p.partial ? min(n_b, kv_begin + p.split_keys) : n_b;
+  // no work: a key chunk past the batch's keys, or a CTA whose rows are all
+  // padding context rows; the epilogue then writes neutral partials / zeros
+  const bool all_pad = p.pad_rows && row0 >= n_b && row0 + kTiles * kQTile <= p.N;
+  const int n_tiles = (all_pad || kv_end <= kv_begin) ? 0 : static_cast<int>((kv_end - kv_begin + kKvTile - 1) / kKvTile);
 
   // ---- set-up
   if (threadIdx.x == 0) {
@@ -456,6 +462,10 @@ __global__ void __launch_bounds__(Cfg<kTiles>::kThreads, Cfg<kTiles>::kMinBlocks
       if (row < p.T) {
         const float lf = __uint_as_float(l);
         if (!p.partial) {
+          // a padding context row of a ragged batch gets zeros (n_b re-read
+          // here rather than kept in registers through the loop)
+          const int64_t nb = p.n_keys != nullptr ? (int64_t)__ldg(p.n_keys + bh / p.H) : p.N;
+          const bool zero = p.pad_rows && row >= nb && row < p.N;
           const int64_t b = bh / p.H, h = bh % p.H;
           uint4* dst = reinterpret_cast<uint4*>(p.out + ((b * p.T + row) * p.H + h) * kHeadDim);
 #pragma unroll
@@ -470,7 +480,7 @@ __global__ void __launch_bounds__(Cfg<kTiles>::kThreads, Cfg<kTiles>::kMinBlocks
                                                 __float2half_rn(__fdiv_rn(__fmul_rn(x1, s_v), lf)));
               w[k] = *reinterpret_cast<const uint32_t*>(&hv);
             }
-            dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[v] = zero ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(w[0], w[1], w[2], w[3]);
           }
         } else {
           const int64_t prow = (split * p.BH + bh) * p.T + row;
@@ -484,6 +494,24 @@ __global__ void __launch_bounds__(Cfg<kTiles>::kThreads, Cfg<kTiles>::kMinBlocks
             dst[8 + v] = make_float4(__uint_as_float(o1[4 * v]), __uint_as_float(o1[4 * v + 1]),
                                      __uint_as_float(o1[4 * v + 2]), __uint_as_float(o1[4 * v + 3]));
           reinterpret_cast<float2*>(p.part_ml)[prow] = make_float2(m2, lf);
+        }
+      }
+    } else if (ok) {
+      // no keys to attend: a padding-only CTA writes zeros; an empty key chunk
+      // writes the neutral partial (acc = 0, m2 = -inf, l = 0: weight 0 in the combine)
+      const int64_t row = row0 + (int64_t)t * kQTile + 32 * wq + lane;
+      if (row < p.T) {
+        if (!p.partial) {
+          const int64_t b = bh / p.H, h = bh % p.H;
+          uint4* dst = reinterpret_cast<uint4*>(p.out + ((b * p.T + row) * p.H + h) * kHeadDim);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+        } else {
+          const int64_t prow = (split * p.BH + bh) * p.T + row;
+          float4* dst = reinterpret_cast<float4*>(p.part_acc + prow * kHeadDim);
+#pragma unroll
+          for (int v = 0; v < 16; ++v) dst[v] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          reinterpret_cast<float2*>(p.part_ml)[prow] = make_float2(-INFINITY, 0.0f);
         }
       }
     }
@@ -617,6 +645,8 @@ cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t
   p.part_acc = a.part_acc;
   p.part_ml = a.part_ml;
   p.err = a.err;
+  p.n_keys = a.n_keys;
+  p.pad_rows = a.pad_rows ? 1 : 0;
   // at most 128 rows (small prediction batches): one query tile per CTA, two CTAs per SM
   if (a.T <= kQTile) return launch_kernel<1>(tq, tk, tv, p, BH, st);
   return launch_kernel<2>(tq, tk, tv, p, BH, st);

@@ -70,6 +70,7 @@ struct HParams {
   int64_t n_pairs;
   __half* out;      // [B][T][H][64]
   uint32_t* err;
+  const int32_t* n_keys;  // [B] keys per batch (rows [n_b, N) are padding), or nullptr: N
 };
 
 __device__ __forceinline__ void raise_abort_h(SmemH& s, uint32_t* err, uint32_t code) {
@@ -130,7 +131,10 @@ __global__ void __launch_bounds__(kThreadsH, 1)
   const int64_t bh = blk / p.n_pairs;
   const int32_t b = static_cast<int32_t>(bh / p.H), h = static_cast<int32_t>(bh % p.H);
   const int64_t row0 = pair * (kTilesH * kQTile);
-  const int n_tiles = static_cast<int>((p.N + kKvTile - 1) / kKvTile);
+  const int64_t n_b = p.n_keys != nullptr ? (int64_t)__ldg(p.n_keys + b) : p.N;  // this batch's keys
+  // a CTA whose rows are all padding context rows only writes zeros
+  const bool all_pad = row0 >= n_b && row0 + kTilesH * kQTile <= p.N;
+  const int n_tiles = all_pad ? 0 : static_cast<int>((n_b + kKvTile - 1) / kKvTile);
 
   if (threadIdx.x == 0) {
     mbar_init(&s.q_full, 1);
@@ -282,7 +286,7 @@ __global__ void __launch_bounds__(kThreadsH, 1)
         break;
       }
       tc_fence_after();
-      const int64_t nvalid = p.N - (int64_t)it * kKvTile;
+      const int64_t nvalid = n_b - (int64_t)it * kKvTile;
       uint32_t r[4][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(t_s + 32 * c, r[c]);
@@ -352,14 +356,17 @@ __global__ void __launch_bounds__(kThreadsH, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok && lane == 0) raise_abort_h(s, p.err, kErrTimeoutO);
     }
-    if (ok && n_tiles > 0) {
-      tc_fence_after();
+    if (ok) {
       uint32_t o0[32], o1[32];
-      tmem_ld_32x32b_x32(t_o, o0);
-      tmem_ld_32x32b_x32(t_o + 32, o1);
-      tmem_ld_wait();
+      if (n_tiles > 0) {
+        tc_fence_after();
+        tmem_ld_32x32b_x32(t_o, o0);
+        tmem_ld_32x32b_x32(t_o + 32, o1);
+        tmem_ld_wait();
+      }
       const int64_t row = row0 + (int64_t)t * kQTile + 32 * wq + lane;
       if (row < p.T) {
+        const bool zero = n_tiles == 0 || (row >= n_b && row < p.N);  // padding context row
         const float lf = ((l[0] + l[1]) + (l[2] + l[3])) + ((l[4] + l[5]) + (l[6] + l[7]));
         uint4* dst = reinterpret_cast<uint4*>(p.out + (((int64_t)b * p.T + row) * p.H + h) * kHeadDim);
 #pragma unroll
@@ -370,7 +377,7 @@ __global__ void __launch_bounds__(kThreadsH, 1)
             const int e = 8 * v + 2 * k;
             const float x0 = __uint_as_float(e < 32 ? o0[e] : o1[e - 32]);
             const float x1 = __uint_as_float(e + 1 < 32 ? o0[e + 1] : o1[e + 1 - 32]);
-            w[k] = f16x2(__fdiv_rn(x0, lf), __fdiv_rn(x1, lf));
+            w[k] = zero ? 0u : f16x2(__fdiv_rn(x0, lf), __fdiv_rn(x1, lf));
           }
           dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
         }
@@ -416,7 +423,8 @@ bool make_map_f16(CUtensorMap* m, const void* base, int rank, const cuuint64_t* 
 }  // namespace
 
 cudaError_t launch_attention_f16(const __half* q_scaled, const __half* k, const __half* vt, int32_t B, int64_t T,
-                                 int64_t N, int32_t H, int64_t ld_v, __half* out, uint32_t* err, cudaStream_t st) {
+                                 int64_t N, int32_t H, int64_t ld_v, const int32_t* n_keys, __half* out,
+                                 uint32_t* err, cudaStream_t st) {
   // Q' [B][T][H][64] and K [B][N][H][64]: 4-D {64, H, rows, B}, box {64, 1, 128, 1}
   const cuuint64_t dq[4] = {64, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
   const cuuint64_t sq[3] = {128, (cuuint64_t)H * 128, (cuuint64_t)T * H * 128};
@@ -440,6 +448,7 @@ cudaError_t launch_attention_f16(const __half* q_scaled, const __half* k, const 
   p.n_pairs = (T + kTilesH * kQTile - 1) / (kTilesH * kQTile);
   p.out = out;
   p.err = err;
+  p.n_keys = n_keys;
   const size_t smem = sizeof(SmemH) + 1024;
   cudaError_t e = cudaFuncSetAttribute(icl_attention_f16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));

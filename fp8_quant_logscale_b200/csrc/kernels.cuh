@@ -27,7 +27,22 @@ struct QScale {
   const float* c_h;    // [H] per-head coefficients (device)
   const __half* gate;  // [B][rows][H] or nullptr (LogScale)
   const __half* gate_w;  // [B][rows][H] precomputed fp16(1 + fp16(tanh g)), or nullptr: evaluate in place
+  const float* lam_b;  // [B] per-batch lam (device; ragged contexts), or nullptr: lam for every batch
 };
+
+// Ragged contexts: batch b has n_b = n_valid[b] unmasked context rows (rows
+// [n_b, N) are padding).  The per-batch lengths and their lam live in device
+// memory right after the [3][B][H] scales ("scales block"): n_b as int32 [B],
+// then lam_b as fp32 [B].
+inline size_t scales_block_words(int64_t B, int64_t H, bool ragged) { return 3 * B * H + (ragged ? 2 * B : 0); }
+constexpr int kMetaChunk = 256;  // batches per meta-writing launch (kernel-parameter payload)
+struct MetaChunk {
+  int32_t b0, count;
+  int32_t n[kMetaChunk];
+  float lam[kMetaChunk];
+};
+// Writes n_b and lam_b of batches [b0, b0 + count) into the scales block's meta words.
+cudaError_t launch_write_meta(const MetaChunk& c, int32_t* n_dst, float* lam_dst, cudaStream_t st);
 
 // Tensor-wide problem description for the elementwise kernels.
 struct RowsDesc {
@@ -37,35 +52,42 @@ struct RowsDesc {
 };
 
 cudaError_t launch_qscale(const __half* q, __half* out, int32_t B, int64_t rows, int32_t H, QScale qs,
-                          cudaStream_t st);
+                          cudaStream_t st);  // qs.lam_b, if set, is indexed by b
 
 // w[i] = fp16(1 + fp16(tanh(gate[i]))) for i < n: the GatedLogScale factor, once per (row, head).
 cudaError_t launch_gate_factors(const __half* gate, int64_t n, __half* w, cudaStream_t st);
 
 // amax words: [3][B][H] uint32 (float bits, values >= 0).  Must be zeroed first.
-cudaError_t launch_context_amax(RowsDesc q, QScale qs, RowsDesc k, RowsDesc v, int64_t n_ctx, uint32_t* amax,
-                                cudaStream_t st);
+// Context rows [0, n_valid ? n_valid[b] : n_ctx) of each batch.
+cudaError_t launch_context_amax(RowsDesc q, QScale qs, RowsDesc k, RowsDesc v, int64_t n_ctx,
+                                const int32_t* n_valid, uint32_t* amax, cudaStream_t st);
 
 // scales[3][B][H] = amax/448 (1 where amax == 0); from the amax words.
 cudaError_t launch_scales_from_amax(const uint32_t* amax, int32_t BH, float* scales, cudaStream_t st);
 
 // Row-major quantisation: dst[b][h][r][64] = e4m3(qscale?(x[b][r][h][:]) / scale[b*H+h]),
-// rows [0, n_rows) of x; dst has dst_rows rows per (b, h).
+// rows [0, n_rows) of x; dst has dst_rows rows per (b, h).  With n_valid, rows
+// [n_valid[b], pad_end) are padding and get zero codes.
 cudaError_t launch_quantize_rows(RowsDesc x, QScale qs, int64_t n_rows, const float* scale, uint8_t* dst,
-                                 int64_t dst_rows, cudaStream_t st);
+                                 int64_t dst_rows, const int32_t* n_valid, int64_t pad_end, cudaStream_t st);
 
-// Transposed quantisation for V: dst[b][h][e][ld] for keys [0, n_ctx), zeros in [n_ctx, ld).
-cudaError_t launch_quantize_vt(RowsDesc v, int64_t n_ctx, const float* scale, uint8_t* dst, int64_t ld,
-                               cudaStream_t st);
+// Transposed quantisation for V: dst[b][h][e][ld] for keys [0, n_b), zeros in
+// [n_b, round_up(n_ctx, 128)); n_b = n_valid ? n_valid[b] : n_ctx.
+cudaError_t launch_quantize_vt(RowsDesc v, int64_t n_ctx, const int32_t* n_valid, const float* scale, uint8_t* dst,
+                               int64_t ld, cudaStream_t st);
 
 // fp16 transpose of V for the normal-precision attention: dst[b][h][e][ld] =
-// v[b][key][h][e] for keys [0, n_ctx), zeros in [n_ctx, round_up(n_ctx, 128)).
-cudaError_t launch_transpose_vt_f16(RowsDesc v, int64_t n_ctx, __half* dst, int64_t ld, cudaStream_t st);
+// v[b][key][h][e] for keys [0, n_b), zeros in [n_b, round_up(n_ctx, 128));
+// n_b = n_valid ? n_valid[b] : n_ctx.
+cudaError_t launch_transpose_vt_f16(RowsDesc v, int64_t n_ctx, const int32_t* n_valid, __half* dst, int64_t ld,
+                                    cudaStream_t st);
 
-// fp16 attention of rows [0, T) of q_scaled [B][T][H][64] to keys [0, N) of
-// k [B][N][H][64] and vt [B][H][64][ld]; out [B][T][H][64] fp16.
+// fp16 attention of rows [0, T) of q_scaled [B][T][H][64] to keys [0, n_b) of
+// k [B][N][H][64] and vt [B][H][64][ld]; out [B][T][H][64] fp16.  With
+// n_keys, n_b = n_keys[b] and rows [n_b, N) (padding) are written as zeros.
 cudaError_t launch_attention_f16(const __half* q_scaled, const __half* k, const __half* vt, int32_t B, int64_t T,
-                                 int64_t N, int32_t H, int64_t ld_v, __half* out, uint32_t* err, cudaStream_t st);
+                                 int64_t N, int32_t H, int64_t ld_v, const int32_t* n_keys, __half* out,
+                                 uint32_t* err, cudaStream_t st);
 
 // ---------------------------------------------------------------- attention
 struct AttnArgs {
@@ -81,6 +103,8 @@ struct AttnArgs {
   float* part_acc;     // split: [S][B*H][T][64]
   float* part_ml;      // split: [S][B*H][T][2] (m2, l)
   uint32_t* err;       // device error word
+  const int32_t* n_keys;  // [B] keys per batch (ragged contexts), or nullptr: N for every batch
+  bool pad_rows;       // rows [n_keys[b], N) are padding context rows: written as zeros
 };
 
 // Builds the tensor maps and launches the tcgen05 attention kernel.

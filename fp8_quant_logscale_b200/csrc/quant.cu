@@ -18,9 +18,11 @@ namespace {
 
 constexpr int kUnroll = 4;  // 16-byte loads in flight per thread
 
-__device__ __forceinline__ float head_scale(const QScale& qs, int h) {
-  // s_h = fp16(c_h * lam): fp32 product, one rounding to the query dtype.
-  return __half2float(__float2half_rn(__fmul_rn(__ldg(qs.c_h + h), qs.lam)));
+__device__ __forceinline__ float head_scale(const QScale& qs, int h, int64_t b) {
+  // s_h = fp16(c_h * lam): fp32 product, one rounding to the query dtype;
+  // lam is the batch's own with ragged contexts.
+  const float lam = qs.lam_b != nullptr ? __ldg(qs.lam_b + b) : qs.lam;
+  return __half2float(__float2half_rn(__fmul_rn(__ldg(qs.c_h + h), lam)));
 }
 
 // w = fp16(1 + fp16(tanh g)); tanh evaluated in double and rounded once to fp16.
@@ -96,7 +98,7 @@ inline int num_sms() {
 
 // ---------------------------------------------------------------- qscale
 __global__ void __launch_bounds__(256) qscale_kernel(const __half* __restrict__ q, __half* __restrict__ out,
-                                                     int64_t n_vec, int H, QScale qs) {
+                                                     int64_t n_vec, int H, int64_t rows, QScale qs) {
   const bool gated = qs.gate != nullptr;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i0 < n_vec; i0 += kUnroll * stride) {
@@ -111,7 +113,7 @@ __global__ void __launch_bounds__(256) qscale_kernel(const __half* __restrict__ 
       const int64_t seg = i >> 3;  // (b*rows + r)*H + h
       const int h = static_cast<int>(seg % H);
       const int64_t br = seg / H;
-      const float s = head_scale(qs, h);
+      const float s = head_scale(qs, h, qs.lam_b != nullptr ? br / rows : 0);
       const float w = gated ? gate_factor(qs, br, H, h) : 1.0f;
       float f[8];
       unpack8(raw[u], f);
@@ -135,7 +137,8 @@ __global__ void __launch_bounds__(256) gate_factor_kernel(const __half* __restri
 // ------------------------------------------------------------ context amax
 // grid: (B * chunks, 3); blockIdx.y selects Q' (query scaling applied), K, V.
 __global__ void context_amax_kernel(RowsDesc q, QScale qs, RowsDesc k, RowsDesc v, int64_t n_ctx,
-                                    int64_t rows_per_cta, int chunks, uint32_t* __restrict__ amax) {
+                                    const int32_t* __restrict__ n_valid, int64_t rows_per_cta, int chunks,
+                                    uint32_t* __restrict__ amax) {
   __shared__ uint32_t s_max[128];
   const int tensor = blockIdx.y;
   const RowsDesc X = tensor == 0 ? q : (tensor == 1 ? k : v);
@@ -149,11 +152,12 @@ __global__ void context_amax_kernel(RowsDesc q, QScale qs, RowsDesc k, RowsDesc 
   const int row_step = blockDim.x / vecs_per_row;
   const int b = blockIdx.x / chunks;
   const int64_t r0 = (blockIdx.x % chunks) * rows_per_cta;
-  const int64_t r1 = min(n_ctx, r0 + rows_per_cta);
+  const int64_t n_b = n_valid != nullptr ? (int64_t)__ldg(n_valid + b) : n_ctx;
+  const int64_t r1 = min(n_b, r0 + rows_per_cta);
   if (t < H) s_max[t] = 0u;
   __syncthreads();
 
-  const float s = do_q ? head_scale(qs, h) : 1.0f;
+  const float s = do_q ? head_scale(qs, h, b) : 1.0f;
   float m = 0.0f;
   for (int64_t r = r0 + t / vecs_per_row; r < r1; r += kUnroll * row_step) {
     uint4 raw[kUnroll];
@@ -193,8 +197,8 @@ __global__ void scales_kernel(const uint32_t* __restrict__ amax, int n, float* _
 
 // ----------------------------------------------------- row-major quantise
 __global__ void quantize_rows_kernel(RowsDesc X, QScale qs, int64_t n_rows, const float* __restrict__ scale,
-                                     uint8_t* __restrict__ dst, int64_t dst_rows, int64_t rows_per_cta,
-                                     int chunks) {
+                                     uint8_t* __restrict__ dst, int64_t dst_rows, const int32_t* __restrict__ n_valid,
+                                     int64_t pad_end, int64_t rows_per_cta, int chunks) {
   const bool do_q = qs.enabled;
   const bool gated = do_q && qs.gate != nullptr;
   const int H = X.H;
@@ -207,8 +211,9 @@ __global__ void quantize_rows_kernel(RowsDesc X, QScale qs, int64_t n_rows, cons
   const int b = blockIdx.x / chunks;
   const int64_t r0 = (blockIdx.x % chunks) * rows_per_cta;
   const int64_t r1 = min(n_rows, r0 + rows_per_cta);
-  const float s = do_q ? head_scale(qs, h) : 1.0f;
+  const float s = do_q ? head_scale(qs, h, b) : 1.0f;
   const Divider dv = make_divider(__ldg(scale + b * H + h));
+  const int64_t pad0 = n_valid != nullptr ? (int64_t)__ldg(n_valid + b) : pad_end;  // padding rows [pad0, pad_end)
   uint8_t* dbase = dst + ((int64_t)b * H + h) * dst_rows * kHeadDim + j * 8;
   for (int64_t r = r0 + t / vecs_per_row; r < r1; r += kUnroll * row_step) {
     uint4 raw[kUnroll];
@@ -232,6 +237,7 @@ __global__ void quantize_rows_kernel(RowsDesc X, QScale qs, int64_t n_rows, cons
       uint2 codes;
       codes.x = e4m3x2(f[0], f[1]) | (e4m3x2(f[2], f[3]) << 16);
       codes.y = e4m3x2(f[4], f[5]) | (e4m3x2(f[6], f[7]) << 16);
+      if (rr >= pad0 && rr < pad_end) codes = make_uint2(0u, 0u);
       *reinterpret_cast<uint2*>(dbase + rr * kHeadDim) = codes;
     }
   }
@@ -240,14 +246,16 @@ __global__ void quantize_rows_kernel(RowsDesc X, QScale qs, int64_t n_rows, cons
 // --------------------------------------------------- transposed V quantise
 // grid: (ld / 128, B*H), 256 threads.  Reads 128 keys x 64 of one head,
 // writes 64 rows of 128 keys (one 128-byte line each) via a padded smem tile.
-__global__ void __launch_bounds__(256) quantize_vt_kernel(RowsDesc V, int64_t n_ctx, const float* __restrict__ scale,
-                                                          uint8_t* __restrict__ dst, int64_t ld) {
+__global__ void __launch_bounds__(256) quantize_vt_kernel(RowsDesc V, int64_t n_ctx, const int32_t* __restrict__ n_valid,
+                                                          const float* __restrict__ scale, uint8_t* __restrict__ dst,
+                                                          int64_t ld) {
   __shared__ uint32_t tile[kHeadDim][33];  // [e][key/4], 132-byte rows: conflict-free
   const int H = V.H;
   const int64_t bh = blockIdx.y;
   const int b = static_cast<int>(bh / H), h = static_cast<int>(bh % H);
   const int64_t r0 = (int64_t)blockIdx.x * kKvTile;
   const Divider dv = make_divider(__ldg(scale + bh));
+  const int64_t n_b = n_valid != nullptr ? (int64_t)__ldg(n_valid + b) : n_ctx;
   const int t = threadIdx.x;
   const int j = t & 7;  // elements 8j..8j+7
   uint8_t* tb = reinterpret_cast<uint8_t*>(&tile[0][0]);
@@ -255,7 +263,7 @@ __global__ void __launch_bounds__(256) quantize_vt_kernel(RowsDesc V, int64_t n_
 #pragma unroll
   for (int i = 0; i < 4; ++i) {  // all loads first: four 16-byte requests in flight
     const int64_t r = r0 + (t >> 3) + 32 * i;
-    if (r < n_ctx)
+    if (r < n_b)
       raws[i] = __ldcs(reinterpret_cast<const uint4*>(V.x + (((int64_t)b * V.rows + r) * H + h) * kHeadDim) + j);
   }
 #pragma unroll
@@ -263,7 +271,7 @@ __global__ void __launch_bounds__(256) quantize_vt_kernel(RowsDesc V, int64_t n_
     const int rl = (t >> 3) + 32 * i;
     const int64_t r = r0 + rl;
     uint32_t lo = 0, hi = 0;
-    if (r < n_ctx) {
+    if (r < n_b) {
       float f[8];
       unpack8(raws[i], f);
       divide8(f, dv);
@@ -292,13 +300,15 @@ __global__ void __launch_bounds__(256) quantize_vt_kernel(RowsDesc V, int64_t n_
 
 // One (b, h) and 128 keys per block: 16-byte row loads of V, a shared-memory
 // transpose, 32-bit stores of 64 rows (one per head element) of 128 keys.
-__global__ void __launch_bounds__(256) transpose_vt_f16_kernel(RowsDesc V, int64_t n_ctx, __half* __restrict__ dst,
-                                                               int64_t ld) {
+__global__ void __launch_bounds__(256) transpose_vt_f16_kernel(RowsDesc V, int64_t n_ctx,
+                                                               const int32_t* __restrict__ n_valid,
+                                                               __half* __restrict__ dst, int64_t ld) {
   __shared__ uint16_t tile[kHeadDim][kKvTile + 2];  // [e][key]; 65-word rows
   const int H = V.H;
   const int64_t bh = blockIdx.y;
   const int b = static_cast<int>(bh / H), h = static_cast<int>(bh % H);
   const int64_t r0 = (int64_t)blockIdx.x * kKvTile;
+  const int64_t n_b = n_valid != nullptr ? (int64_t)__ldg(n_valid + b) : n_ctx;
   const int t = threadIdx.x;
   const int j = t & 7;  // elements 8j..8j+7
   uint4 raws[4];
@@ -306,7 +316,7 @@ __global__ void __launch_bounds__(256) transpose_vt_f16_kernel(RowsDesc V, int64
   for (int i = 0; i < 4; ++i) {
     const int64_t r = r0 + (t >> 3) + 32 * i;
     raws[i] = make_uint4(0u, 0u, 0u, 0u);
-    if (r < n_ctx)
+    if (r < n_b)
       raws[i] = __ldcs(reinterpret_cast<const uint4*>(V.x + (((int64_t)b * V.rows + r) * H + h) * kHeadDim) + j);
   }
 #pragma unroll
@@ -330,12 +340,26 @@ __global__ void __launch_bounds__(256) transpose_vt_f16_kernel(RowsDesc V, int64
   }
 }
 
+__global__ void write_meta_kernel(MetaChunk c, int32_t* __restrict__ n_dst, float* __restrict__ lam_dst) {
+  const int i = threadIdx.x;
+  if (i < c.count) {
+    n_dst[c.b0 + i] = c.n[i];
+    lam_dst[c.b0 + i] = c.lam[i];
+  }
+}
+
 }  // namespace
 
-cudaError_t launch_transpose_vt_f16(RowsDesc v, int64_t n_ctx, __half* dst, int64_t ld, cudaStream_t st) {
+cudaError_t launch_transpose_vt_f16(RowsDesc v, int64_t n_ctx, const int32_t* n_valid, __half* dst, int64_t ld,
+                                    cudaStream_t st) {
   dim3 grid(static_cast<unsigned>((n_ctx + kKvTile - 1) / kKvTile), static_cast<unsigned>(v.B * v.H));
   if (grid.x == 0) return cudaSuccess;
-  transpose_vt_f16_kernel<<<grid, 256, 0, st>>>(v, n_ctx, dst, ld);
+  transpose_vt_f16_kernel<<<grid, 256, 0, st>>>(v, n_ctx, n_valid, dst, ld);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_write_meta(const MetaChunk& c, int32_t* n_dst, float* lam_dst, cudaStream_t st) {
+  write_meta_kernel<<<1, kMetaChunk, 0, st>>>(c, n_dst, lam_dst);
   return cudaGetLastError();
 }
 
@@ -345,7 +369,7 @@ cudaError_t launch_qscale(const __half* q, __half* out, int32_t B, int64_t rows,
   if (n_vec == 0) return cudaSuccess;
   const int64_t want = (n_vec + 256 * kUnroll - 1) / (256 * kUnroll);
   const int grid = static_cast<int>(want < (int64_t)num_sms() * 8 ? want : (int64_t)num_sms() * 8);
-  qscale_kernel<<<grid, 256, 0, st>>>(q, out, n_vec, H, qs);
+  qscale_kernel<<<grid, 256, 0, st>>>(q, out, n_vec, H, rows, qs);
   return cudaGetLastError();
 }
 
@@ -357,8 +381,8 @@ cudaError_t launch_gate_factors(const __half* gate, int64_t n, __half* w, cudaSt
   return cudaGetLastError();
 }
 
-cudaError_t launch_context_amax(RowsDesc q, QScale qs, RowsDesc k, RowsDesc v, int64_t n_ctx, uint32_t* amax,
-                                cudaStream_t st) {
+cudaError_t launch_context_amax(RowsDesc q, QScale qs, RowsDesc k, RowsDesc v, int64_t n_ctx,
+                                const int32_t* n_valid, uint32_t* amax, cudaStream_t st) {
   const int threads = row_threads(q.H);
   const int rows_per_pass = threads / (8 * q.H);
   // about 8 CTAs per SM over the three tensors
@@ -367,7 +391,8 @@ cudaError_t launch_context_amax(RowsDesc q, QScale qs, RowsDesc k, RowsDesc v, i
   rows_per_cta = ((rows_per_cta + rows_per_pass - 1) / rows_per_pass) * rows_per_pass;
   chunks = (n_ctx + rows_per_cta - 1) / rows_per_cta;
   dim3 grid(static_cast<unsigned>(q.B * chunks), 3);
-  context_amax_kernel<<<grid, threads, 0, st>>>(q, qs, k, v, n_ctx, rows_per_cta, static_cast<int>(chunks), amax);
+  context_amax_kernel<<<grid, threads, 0, st>>>(q, qs, k, v, n_ctx, n_valid, rows_per_cta, static_cast<int>(chunks),
+                                                amax);
   return cudaGetLastError();
 }
 
@@ -378,7 +403,7 @@ cudaError_t launch_scales_from_amax(const uint32_t* amax, int32_t BH, float* sca
 }
 
 cudaError_t launch_quantize_rows(RowsDesc x, QScale qs, int64_t n_rows, const float* scale, uint8_t* dst,
-                                 int64_t dst_rows, cudaStream_t st) {
+                                 int64_t dst_rows, const int32_t* n_valid, int64_t pad_end, cudaStream_t st) {
   if (n_rows == 0) return cudaSuccess;
   const int threads = row_threads(x.H);
   const int rows_per_pass = threads / (8 * x.H);
@@ -387,14 +412,14 @@ cudaError_t launch_quantize_rows(RowsDesc x, QScale qs, int64_t n_rows, const fl
   rows_per_cta = ((rows_per_cta + rows_per_pass - 1) / rows_per_pass) * rows_per_pass;
   chunks = (n_rows + rows_per_cta - 1) / rows_per_cta;
   quantize_rows_kernel<<<static_cast<unsigned>(x.B * chunks), threads, 0, st>>>(
-      x, qs, n_rows, scale, dst, dst_rows, rows_per_cta, static_cast<int>(chunks));
+      x, qs, n_rows, scale, dst, dst_rows, n_valid, pad_end, rows_per_cta, static_cast<int>(chunks));
   return cudaGetLastError();
 }
 
-cudaError_t launch_quantize_vt(RowsDesc v, int64_t n_ctx, const float* scale, uint8_t* dst, int64_t ld,
-                               cudaStream_t st) {
+cudaError_t launch_quantize_vt(RowsDesc v, int64_t n_ctx, const int32_t* n_valid, const float* scale, uint8_t* dst,
+                               int64_t ld, cudaStream_t st) {
   dim3 grid(static_cast<unsigned>(ld / kKvTile), static_cast<unsigned>(v.B * v.H));
-  quantize_vt_kernel<<<grid, 256, 0, st>>>(v, n_ctx, scale, dst, ld);
+  quantize_vt_kernel<<<grid, 256, 0, st>>>(v, n_ctx, n_valid, scale, dst, ld);
   return cudaGetLastError();
 }
 

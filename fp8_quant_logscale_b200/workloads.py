@@ -22,7 +22,8 @@ from concurrent.futures import ThreadPoolExecutor
 import numpy as np
 
 _CHUNK = 1 << 22
-_TENSOR_IDS = {"q": 1, "k": 2, "v": 3, "gate": 4, "c_h": 5, "head_factor": 6, "outlier": 7, "queries": 8}
+_TENSOR_IDS = {"q": 1, "k": 2, "v": 3, "gate": 4, "c_h": 5, "head_factor": 6, "outlier": 7, "queries": 8,
+               "ctx_len": 9}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -38,6 +39,7 @@ class Workload:
     outliers: float = 0.0  # fraction of elements multiplied by outlier_scale
     outlier_scale: float = 20.0
     cached: bool = False   # cached prediction against an n_ctx-row cache
+    ragged: tuple | None = None  # batch b has n_b ~ U{floor(lo*N)+1 .. floor(hi*N)} unmasked context rows
     seed: int = 0
     description: str = ""
 
@@ -66,6 +68,11 @@ WORKLOADS = {
         description="N=8192, M=1024, H=8, d=64, fp16 N(0,1) scaled per (tensor, head) by U(0.5,4); "
                     "GatedLogScale; at most 8,192 context rows (or the final layer): normal-precision fp16 "
                     "attention"),
+    "ragged_b16_n16k_m1k_h8": Workload(
+        "ragged_b16_n16k_m1k_h8", 16384, 1024, 8, batch=16, ragged=(0.5, 1.0), seed=7,
+        description="16 estimators in one batch, padded to N=16384 context rows, each with n_b ~ "
+                    "U{8193..16384} unmasked rows; M=1024 queries, H=8, d=64, fp16 N(0,1); LogScale with "
+                    "n = n_b; padding rows hold random values the layer must ignore"),
     "cached_n512k_m1k_h8": Workload(
         "cached_n512k_m1k_h8", 524288, 1024, 8, cached=True, seed=5,
         description="M=1024 fp16 N(0,1) queries, H=8, d=64, LogScale n=524288, against a resident FP8 "
@@ -141,7 +148,13 @@ def make_inputs(w: Workload, seed: int | None = None, n_ctx: int | None = None, 
         gate = np.empty((B, N + M, H), np.float32)
         _normal_fill(gate, s, "gate")
         gate = gate.astype(np.float16)
-    out = dict(workload=w, q=q, k=k, v=v, c_h=c_h, gate=gate, B=B, N=N, M=M, H=H, d=d)
+    ctx_len = None
+    if w.ragged is not None:
+        lo = max(1, int(np.floor(w.ragged[0] * N)) + 1)
+        hi = max(lo, int(np.floor(w.ragged[1] * N)))
+        g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([s, _TENSOR_IDS["ctx_len"]])))
+        ctx_len = g.integers(lo, hi + 1, size=B).astype(np.int64)
+    out = dict(workload=w, q=q, k=k, v=v, c_h=c_h, gate=gate, B=B, N=N, M=M, H=H, d=d, ctx_len=ctx_len)
     if w.cached:
         qq = np.empty((B, M, H, d), np.float32)
         _normal_fill(qq, s, "queries")

@@ -75,12 +75,15 @@ typedef enum {
  * FP8 K/V cache: the fitted state that cached prediction reads (the analogue
  * of the pages' quantised KV cache entry).  The caller allocates the three
  * buffers with the sizes from sdm_cache_layout() on one device and fills in
- * every field; sdm_fp8_quantize_context() or sdm_icl_attention() writes the
- * contents and sets `filled` to 1.
- *   k8     [B][H][N][64]   e4m3, keys row-major
+ * every field; sdm_fp8_quantize_context(), sdm_icl_attention() or
+ * sdm_icl_attention_ragged() writes the contents and sets `filled` to 1 and
+ * `ragged` to 0 or 1 (initialise both to 0).
+ *   k8     [B][H][N][64]   e4m3, keys row-major (rows past n_b: zero codes)
  *   v8t    [B][H][64][ld_v] e4m3, V transposed (keys contiguous);
- *          ld_v = N rounded up to a multiple of 128; keys [N, ld_v) are zero
- *   scales [3][B][H]        fp32: s_q, s_k, s_v (amax/448 over context rows)
+ *          ld_v = N rounded up to a multiple of 128; keys [n_b, ld_v) are zero
+ *   scales the scales block, fp32 words: [3][B][H] s_q, s_k, s_v (amax/448
+ *          over the context rows), then, for a ragged cache, n_b as int32 [B]
+ *          and fp32 ln(n_b) [B]; size from sdm_cache_layout()
  */
 typedef struct {
   uint8_t* k8;
@@ -93,6 +96,7 @@ typedef struct {
   int32_t head_dim;
   int32_t device;
   int32_t filled;
+  int32_t ragged; /* 1: per-batch context lengths n_b are stored in the scales block */
 } sdm_fp8_cache;
 
 /* Human-readable name of a status code (static storage). */
@@ -194,6 +198,24 @@ sdm_status sdm_icl_attention(const void* q, const void* k, const void* v, int32_
                              void* out, sdm_fp8_cache* cache, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Batched estimators with ragged contexts ("unmasked context rows",
+ * "[FP8 3/4] ...", opening section): batch b has n_b = ctx_len[b] context
+ * rows (1 <= n_b <= N); its rows [n_b, N) are padding.  Each batch is the
+ * layer of sdm_icl_attention on its own unmasked rows: query scaling with
+ * n = n_b, scales from rows [0, n_b) only, context rows [0, n_b) and query
+ * rows [N, T) attend to keys [0, n_b).  Padding rows never reach a scale or a
+ * softmax (their contents, NaN included, cannot change a result) and their
+ * outputs are written as zeros.
+ *   ctx_len  HOST array of B int64 (read during the call; not kept)
+ *   other arguments as sdm_icl_attention; a cache given here is marked ragged
+ *   and keeps n_b, so sdm_cached_attention masks and scales by batch.
+ */
+sdm_status sdm_icl_attention_ragged(const void* q, const void* k, const void* v, int32_t batch, int64_t n_ctx,
+                                    int64_t n_query, int32_t heads, int32_t head_dim, const int64_t* ctx_len,
+                                    const float* c_h, const void* gate, void* out, sdm_fp8_cache* cache, void* ws,
+                                    size_t ws_bytes, void* stream);
+
+/*
  * Step 4 -- cached prediction ("model.predict(queries)" after "model.fit" on
  * "[FP8 3/4] ...").  The M query rows are query-scaled with n = cache->n_ctx,
  * quantised with the cache's context-derived s_q, and attend to the cache's
@@ -202,6 +224,8 @@ sdm_status sdm_icl_attention(const void* q, const void* k, const void* v, int32_
  *   q    [B][M][H][d] fp16 raw;  gate [B][M][H] fp16 or NULL;  c_h [H] fp32
  *   out  [B][M][H][d] fp16
  *   ws   >= sdm_workspace_size(SDM_OP_CACHED_ATTENTION, B, cache->n_ctx, M, ...)
+ * With a ragged cache, batch b's queries are scaled with n = n_b and attend to
+ * its keys [0, n_b).
  * Returns SDM_ERR_CACHE_MISMATCH if the cache is unfilled, on another device,
  * or its batch/heads/head_dim differ from the call's.
  */
@@ -241,6 +265,13 @@ int32_t sdm_fp8_eligible(int64_t n_unmasked_ctx, int32_t final_layer);
 sdm_status sdm_icl_attention_f16(const void* q, const void* k, const void* v, int32_t batch, int64_t n_ctx,
                                  int64_t n_query, int32_t heads, int32_t head_dim, const float* c_h,
                                  const void* gate, void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* sdm_icl_attention_f16 with ragged contexts: ctx_len as for
+ * sdm_icl_attention_ragged (host array, 1 <= n_b <= N); padding rows out 0. */
+sdm_status sdm_icl_attention_f16_ragged(const void* q, const void* k, const void* v, int32_t batch, int64_t n_ctx,
+                                        int64_t n_query, int32_t heads, int32_t head_dim, const int64_t* ctx_len,
+                                        const float* c_h, const void* gate, void* out, void* ws, size_t ws_bytes,
+                                        void* stream);
 
 /*
  * Step 2 without a workspace.  This entry point has no counterpart in the

@@ -238,3 +238,61 @@ def layer(q, k, v, n_ctx: int, c_h, gate=None, rows=None, split: int = 0, delta:
     o16, o, allow = attention(q8, k8, v8, s_q, s_k, s_v, rows=rows, split=split, delta=delta)
     return dict(q_scaled=qs, s_q=s_q, s_k=s_k, s_v=s_v, q8=q8, k8=k8, v8=v8,
                 out16=o16, out=o, allow=allow)
+
+
+# --- ragged batches (batched estimators with padded contexts) ------------------
+
+def _ragged_rows(n_b: int, N: int, T: int) -> np.ndarray:
+    """Rows of a padded batch that the layer computes: context [0, n_b) and queries [N, T)."""
+    return np.concatenate([np.arange(n_b), np.arange(N, T)]).astype(np.int64)
+
+
+def layer_ragged(q, k, v, ctx_len, c_h, gate=None, split: int = 0, delta: float = 0.0):
+    """A batch of estimators whose contexts are padded to N rows ("unmasked context
+    rows", [FP8 3/4] opening section): batch b is `layer` on its own rows only --
+    query scaling with n = n_b, scales from rows [0, n_b), context rows [0, n_b)
+    and query rows [N, T) attending to keys [0, n_b).  Padding rows [n_b, N) take
+    part in nothing; their outputs and e4m3 codes are zero.
+
+    q [B,T,H,d], k/v [B,N,H,d] fp16, ctx_len [B] with 1 <= n_b <= N.
+    Returns out16/out/allow [B,T,H,d], s_q/s_k/s_v [B,H], q8 [B,H,T,d], k8/v8 [B,H,N,d]
+    and q_scaled [B,T,H,d] (padding rows zero).
+    """
+    B, T, H, d = q.shape
+    N = k.shape[1]
+    ctx_len = [int(x) for x in ctx_len]
+    assert len(ctx_len) == B and all(1 <= n <= N for n in ctx_len)
+    res = dict(out16=np.zeros((B, T, H, d), np.float16), out=np.zeros((B, T, H, d)),
+               allow=np.zeros((B, T, H, d)), s_q=np.empty((B, H), np.float32), s_k=np.empty((B, H), np.float32),
+               s_v=np.empty((B, H), np.float32), q8=np.zeros((B, H, T, d), np.uint8),
+               k8=np.zeros((B, H, N, d), np.uint8), v8=np.zeros((B, H, N, d), np.uint8),
+               q_scaled=np.zeros((B, T, H, d), np.float16))
+    for b, n in enumerate(ctx_len):
+        rows = _ragged_rows(n, N, T)
+        g = None if gate is None else np.ascontiguousarray(gate[b:b + 1, rows])
+        r = layer(np.ascontiguousarray(q[b:b + 1, rows]), np.ascontiguousarray(k[b:b + 1, :n]),
+                  np.ascontiguousarray(v[b:b + 1, :n]), n, c_h, g, split=split, delta=delta)
+        for key in ("out16", "out", "allow", "q_scaled"):
+            res[key][b, rows] = r[key][0]
+        for key in ("s_q", "s_k", "s_v"):
+            res[key][b] = r[key][0]
+        res["q8"][b][:, rows] = r["q8"][0]
+        res["k8"][b][:, :n] = r["k8"][0]
+        res["v8"][b][:, :n] = r["v8"][0]
+    return res
+
+
+def attention_exact_ragged(q, k, v, ctx_len, rows=None):
+    """Double-precision attention of a padded batch: row i of batch b attends to keys
+    [0, n_b); rows [n_b, N) are padding (0).  q [B,T,H,d] (already query-scaled), k/v
+    [B,N,H,d].  Returns [B,n,H,d] f64 for the selected rows (all rows if None)."""
+    B, T, H, d = q.shape
+    N = k.shape[1]
+    rows = np.arange(T, dtype=np.int64) if rows is None else np.asarray(rows, np.int64)
+    out = np.zeros((B, rows.size, H, d))
+    for b, n in enumerate(int(x) for x in ctx_len):
+        sel = np.nonzero((rows < n) | (rows >= N))[0]
+        if sel.size:
+            out[b, sel] = attention_exact(np.ascontiguousarray(q[b:b + 1]), np.ascontiguousarray(k[b:b + 1, :n]),
+                                          np.ascontiguousarray(v[b:b + 1, :n]), rows=rows[sel])[0]
+    return out

@@ -42,14 +42,14 @@ def test_every_declared_symbol_is_exported(L):
 def test_status_strings(L):
     for code, name in binding.STATUS_NAMES.items():
         assert L.sdm_status_string(code).decode().startswith(name)
-    assert L.sdm_version() == 100
+    assert L.sdm_version() == 101
 
 
 def test_cache_layout_and_workspace_sizes(L):
     kb, vb, sb, ld = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_int64()
     st = L.sdm_cache_layout(2, 1000, 3, 64, ctypes.byref(kb), ctypes.byref(vb), ctypes.byref(sb), ctypes.byref(ld))
     assert st == 0 and ld.value == 1024
-    assert kb.value == 2 * 3 * 1000 * 64 and vb.value == 2 * 3 * 64 * 1024 and sb.value == 3 * 2 * 3 * 4
+    assert kb.value == 2 * 3 * 1000 * 64 and vb.value == 2 * 3 * 64 * 1024 and sb.value == (3 * 2 * 3 + 2 * 2) * 4  # scales + ragged meta
     assert L.sdm_cache_layout(1, 1000, 3, 32, None, None, None, None) == 2       # d != 64
     assert L.sdm_cache_layout(1, 0, 3, 64, None, None, None, None) == 1          # N < 1
     assert L.sdm_cache_layout(1, 10, 129, 64, None, None, None, None) == 2       # too many heads
@@ -105,3 +105,17 @@ def test_f16_workspace_and_shape_errors(L):
     assert L.sdm_icl_attention_f16(None, None, None, 1, 0, 5, 4, 64, None, None, None, None, 0, None) == 1
     assert L.sdm_icl_attention_f16(None, None, None, 1, 10, 5, 4, 48, None, None, None, None, 0, None) == 2
     assert L.sdm_icl_attention_f16(None, None, None, 1, 10, 5, 200, 64, None, None, None, None, 0, None) == 2
+
+
+def test_ragged_argument_errors(L):
+    import ctypes as C
+    lens = lambda *x: (C.c_int64 * len(x))(*x)
+    f = L.sdm_icl_attention_ragged
+    assert f(None, None, None, 2, 100, 5, 4, 64, None, None, None, None, None, None, 0, None) == 1   # no ctx_len
+    assert f(None, None, None, 2, 100, 5, 4, 64, lens(100, 0), None, None, None, None, None, 0, None) == 1
+    assert f(None, None, None, 2, 100, 5, 4, 64, lens(101, 50), None, None, None, None, None, 0, None) == 1
+    g = L.sdm_icl_attention_f16_ragged
+    assert g(None, None, None, 2, 100, 5, 4, 64, None, None, None, None, None, 0, None) == 1
+    assert g(None, None, None, 2, 100, 5, 4, 64, lens(-3, 7), None, None, None, None, 0, None) == 1
+    if not torch.cuda.is_available():  # valid lengths get past the host checks to the device query
+        assert f(None, None, None, 2, 100, 5, 4, 64, lens(100, 1), None, None, None, None, None, 0, None) == 7
