@@ -415,6 +415,18 @@ def run_per_kernel(args):
         ]
     # a filled cache and Q8 for the attention steps
     q8.copy_(sdm.fp8_quantize_context(sdm.qscale_fused(q, c_h, N, gate), k, v, N, cache=cache)[0])
+    # the same cache with K8 / V8^T in page-locked host memory, and the host link it is read over
+    off = cache.offload()
+    ws_o = sdm.new_workspace(sdm.workspace_size(binding.OP_CACHED_ATTENTION_OFFLOAD, B, N, Mq, H), device)
+    k_dst, v_dst = torch.empty_like(cache.k8), torch.empty_like(cache.v8t)
+    cache_bytes = off.k8.numel() + off.v8t.numel()
+    steps += [
+        ("a8 cached prediction from the host-offloaded cache, 1024 queries (sdm_cached_attention_offload)",
+         lambda: sdm.cached_attention_offload(queries, off, c_h, out=pred, ws=ws_o),
+         cache_bytes + 2 * el(Mq) * 2, B * attn_flops(Mq, N, H)),
+        ("ref: page-locked host-to-device copy of the same K8 / V8^T bytes (cudaMemcpyAsync, not this library)",
+         lambda: (k_dst.copy_(off.k8, non_blocking=True), v_dst.copy_(off.v8t, non_blocking=True)), cache_bytes, 0.0),
+    ]
     for name, fn, nbytes, flops in steps:
         times = []
         for i in range(args.warmup + args.steps):

@@ -7,10 +7,11 @@ cached prediction over a resident FP8 K/V cache; plus the normal-precision
 (fp16 tcgen05) attention that the precision rule keeps for the final layer and
 short contexts.
 """
-from .binding import (FP8Cache, SdmError, cached_attention, fp8_attention, fp8_eligible, fp8_quantize_context,
-                      icl_attention, icl_attention_f16, icl_layer, lib, new_workspace, qscale_fused, sync_status,
-                      workspace_size)
+from .binding import (FP8Cache, OffloadedFP8Cache, SdmError, cached_attention, cached_attention_offload,
+                      fp8_attention, fp8_eligible, fp8_quantize_context, icl_attention, icl_attention_f16, icl_layer,
+                      lib, new_workspace, qscale_fused, sync_status, workspace_size)
 
-__all__ = ["FP8Cache", "SdmError", "cached_attention", "fp8_attention", "fp8_eligible", "fp8_quantize_context",
+__all__ = ["FP8Cache", "OffloadedFP8Cache", "SdmError", "cached_attention", "cached_attention_offload",
+           "fp8_attention", "fp8_eligible", "fp8_quantize_context",
            "icl_attention", "icl_attention_f16", "icl_layer", "lib", "new_workspace", "qscale_fused", "sync_status",
            "workspace_size"]

@@ -19,6 +19,7 @@ STATUS_NAMES = {0: "SDM_OK", 1: "SDM_ERR_INVALID_ARG", 2: "SDM_ERR_UNSUPPORTED",
                 4: "SDM_ERR_DEVICE_MISMATCH", 5: "SDM_ERR_CACHE_MISMATCH", 6: "SDM_ERR_TIMEOUT",
                 7: "SDM_ERR_CUDA"}
 OP_QUANTIZE_CONTEXT, OP_ICL_ATTENTION, OP_CACHED_ATTENTION, OP_ICL_ATTENTION_F16 = 0, 1, 2, 3
+OP_CACHED_ATTENTION_OFFLOAD = 4
 FP8_MIN_CONTEXT = 8192
 KV_TILE = 128
 HEAD_DIM = 64
@@ -27,7 +28,8 @@ HEAD_DIM = 64
 EXPORTS = ("sdm_status_string", "sdm_version", "sdm_split_keys", "sdm_cache_layout", "sdm_workspace_size", "sdm_qscale_fused",
            "sdm_fp8_quantize_context", "sdm_fp8_quantize_context_noalloc", "sdm_fp8_attention", "sdm_icl_attention",
            "sdm_cached_attention", "sdm_fp8_eligible", "sdm_icl_attention_f16", "sdm_icl_attention_ragged",
-           "sdm_icl_attention_f16_ragged", "sdm_sync_status", "sdm_selftest_wait_timeout")
+           "sdm_icl_attention_f16_ragged", "sdm_cached_attention_offload", "sdm_sync_status",
+           "sdm_selftest_wait_timeout")
 NOALLOC_MAX_BATCH_HEADS = 4096
 
 
@@ -89,6 +91,9 @@ def lib() -> ctypes.CDLL:
         L.sdm_icl_attention_f16_ragged.restype = ctypes.c_int
         L.sdm_icl_attention_f16_ragged.argtypes = [_P, _P, _P, _I32, _I64, _I64, _I32, _I32, _P, _P, _P, _P,
                                                    _P, _SZ, _P]
+        L.sdm_cached_attention_offload.restype = ctypes.c_int
+        L.sdm_cached_attention_offload.argtypes = [_P, _I32, _I64, _I32, _I32, ctypes.POINTER(CacheStruct), _P, _P,
+                                                   _P, _P, _SZ, _P, _P]
         L.sdm_fp8_eligible.restype = _I32
         L.sdm_fp8_eligible.argtypes = [_I64, _I32]
         L.sdm_icl_attention_f16.restype = ctypes.c_int
@@ -191,6 +196,10 @@ class FP8Cache:
     @property
     def ragged(self) -> bool:
         return self.struct.ragged == 1
+
+    def offload(self) -> "OffloadedFP8Cache":
+        """A copy of this (filled) cache with K8 / V8^T in page-locked host memory."""
+        return OffloadedFP8Cache(self)
 
     def ctx_len(self) -> list[int]:
         """Per-batch context lengths (n_ctx for every batch unless the fit was ragged)."""
@@ -385,3 +394,54 @@ def icl_layer(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_ctx: int, c_h
         raise ValueError("an FP8 cache is filled only by an FP8-eligible layer "
                          f"(unmasked context rows={n_unmasked}, final_layer={final_layer})")
     return icl_attention_f16(q, k, v, n_ctx, c_h, gate=gate, out=out, ctx_len=ctx_len)
+
+
+class OffloadedFP8Cache:
+    """An FP8 cache whose K8 / V8^T live in page-locked host memory; the scales block (a few
+    KB) stays on the device.  Read by cached_attention_offload one split-KV chunk at a time."""
+
+    def __init__(self, cache: FP8Cache):
+        if not cache.filled:
+            raise ValueError("only a filled cache can be offloaded")
+        torch.cuda.current_stream(cache.k8.device).synchronize()
+        self.k8 = torch.empty(cache.k8.shape, dtype=torch.uint8, pin_memory=True)
+        self.v8t = torch.empty(cache.v8t.shape, dtype=torch.uint8, pin_memory=True)
+        self.k8.copy_(cache.k8)
+        self.v8t.copy_(cache.v8t)
+        self.block = cache.block.clone()
+        c = cache.struct
+        self.struct = CacheStruct(self.k8.data_ptr(), self.v8t.data_ptr(), self.block.data_ptr(), c.n_ctx, c.ld_v,
+                                  c.batch, c.heads, c.head_dim, c.device, c.filled, c.ragged)
+        self.device = cache.k8.device
+        self.n_ctx = int(c.n_ctx)
+
+
+_copy_streams: dict = {}
+
+
+def cached_attention_offload(q: torch.Tensor, cache: OffloadedFP8Cache, c_h: torch.Tensor,
+                             gate: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                             ws: torch.Tensor | None = None, copy_stream=None) -> torch.Tensor:
+    """Cached prediction against an offloaded cache: q [B,M,H,64] raw fp16 -> out [B,M,H,64] fp16,
+    identical to cached_attention on the same cache.  Host-to-device copies run on copy_stream
+    (default: one side stream per device), overlapped with the attention."""
+    _want(q, torch.float16, "q", 4)
+    _want(c_h, torch.float32, "c_h", 1)
+    if gate is not None:
+        _want(gate, torch.float16, "gate", 3)
+    B, M, H, d = q.shape
+    dev = q.device
+    out = torch.empty_like(q) if out is None else out
+    need = workspace_size(OP_CACHED_ATTENTION_OFFLOAD, B, cache.n_ctx, M, H)
+    ws = new_workspace(need, dev) if ws is None else ws
+    if copy_stream is None:
+        key = dev.index if dev.index is not None else torch.cuda.current_device()
+        if key not in _copy_streams:
+            _copy_streams[key] = torch.cuda.Stream(device=dev)
+        copy_stream = _copy_streams[key]
+    with torch.cuda.device(dev):
+        _check(lib().sdm_cached_attention_offload(_ptr(q), B, M, H, d, ctypes.byref(cache.struct), _ptr(c_h),
+                                                  _ptr(gate), _ptr(out), _ptr(ws), ws.numel(), _stream(dev),
+                                                  ctypes.c_void_p(copy_stream.cuda_stream)),
+               "sdm_cached_attention_offload")
+    return out

@@ -44,6 +44,19 @@ bool on_device(const void* p, int dev) {
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// True if p is page-locked host memory (or device memory of `dev`): what an
+// asynchronous copy can read without staging through the driver.
+bool pinned_or_device(const void* p, int dev) {
+  if (p == nullptr) return false;
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (at.type == cudaMemoryTypeHost) return true;
+  return (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) && at.device == dev;
+}
+
 sdm_status check_shape(int32_t B, int64_t rows_a, int64_t rows_b, int32_t H, int32_t d) {
   if (B < 1 || H < 1 || rows_a < 0 || rows_b < 0) return SDM_ERR_INVALID_ARG;
   if (d != kHeadDim) return SDM_ERR_UNSUPPORTED;
@@ -78,6 +91,7 @@ sdm_status check_tensor(const void* p, int dev) {
 struct WsLayout {
   size_t amax = 0, gate_w = 0, q8 = 0, k8 = 0, v8t = 0, scales = 0, part_acc = 0, part_ml = 0, total = 0;
   size_t q16 = 0, vt16 = 0, meta = 0;  // normal-precision path: q', V^T in fp16, ragged meta
+  size_t stage = 0, stage_bytes = 0;    // offloaded cache: two staging slots of one chunk each
 };
 
 int64_t n_splits_for(int64_t n_ctx) {
@@ -106,7 +120,7 @@ WsLayout ws_layout(sdm_op op, int32_t B, int64_t N, int64_t M, int32_t H, int32_
     w.total = off;
     return w;
   }
-  const int64_t rows = (op == SDM_OP_ICL_ATTENTION) ? N + M : M;
+  const int64_t rows = (op == SDM_OP_ICL_ATTENTION) ? N + M : M;  // cached ops: the M query rows
   w.gate_w = off;  // GatedLogScale factors, one fp16 per (row, head)
   off = align_up(off + BH * (size_t)rows * sizeof(uint16_t), kAlign);
   w.q8 = off;
@@ -120,12 +134,19 @@ WsLayout ws_layout(sdm_op op, int32_t B, int64_t N, int64_t M, int32_t H, int32_
     w.scales = off;  // scales block: [3][B][H] scales, then the ragged meta words
     off = align_up(off + scales_block_words(B, H, true) * sizeof(float), kAlign);
   }
-  if (op == SDM_OP_CACHED_ATTENTION) {
+  if (op == SDM_OP_CACHED_ATTENTION || op == SDM_OP_CACHED_ATTENTION_OFFLOAD) {
     const size_t S = (size_t)n_splits_for(N);
     w.part_acc = off;
     off = align_up(off + S * BH * (size_t)M * kHeadDim * sizeof(float), kAlign);
     w.part_ml = off;
     off = align_up(off + S * BH * (size_t)M * 2 * sizeof(float), kAlign);
+  }
+  if (op == SDM_OP_CACHED_ATTENTION_OFFLOAD) {
+    // one chunk of split_keys_for(N) keys per slot: K8 [B][H][L][64] + V8^T [B][H][64][L]
+    const size_t L = (size_t)split_keys_for(N);
+    w.stage_bytes = align_up(2 * BH * L * kHeadDim, kAlign);
+    w.stage = off;
+    off += 2 * w.stage_bytes;
   }
   w.total = off;
   return w;
@@ -274,7 +295,7 @@ sdm_status sdm_cache_layout(int32_t B, int64_t N, int32_t H, int32_t d, size_t* 
 
 size_t sdm_workspace_size(sdm_op op, int32_t B, int64_t N, int64_t M, int32_t H, int32_t d, int32_t keep_cache) {
   if (op != SDM_OP_QUANTIZE_CONTEXT && op != SDM_OP_ICL_ATTENTION && op != SDM_OP_CACHED_ATTENTION &&
-      op != SDM_OP_ICL_ATTENTION_F16)
+      op != SDM_OP_ICL_ATTENTION_F16 && op != SDM_OP_CACHED_ATTENTION_OFFLOAD)
     return 0;
   if (check_shape(B, N, M, H, d) != SDM_OK || N < 1) return 0;
   return ws_layout(op, B, N, M, H, keep_cache).total;
@@ -574,6 +595,124 @@ sdm_status sdm_icl_attention_f16_ragged(const void* q, const void* k, const void
 }
 
 
+
+sdm_status sdm_cached_attention_offload(const void* q, int32_t B, int64_t M, int32_t H, int32_t d,
+                                        const sdm_fp8_cache* cache, const float* c_h, const void* gate, void* out,
+                                        void* ws, size_t ws_bytes, void* stream, void* copy_stream) {
+  if (cache == nullptr) return SDM_ERR_INVALID_ARG;
+  SDM_TRY(check_shape(B, cache->n_ctx, M, H, d));
+  const int dev = current_device();
+  if (dev < 0) return SDM_ERR_CUDA;
+  // the cache: K8 / V8^T in page-locked host memory (or on this device), scales block here
+  if (cache->batch != B || cache->heads != H || cache->head_dim != d || cache->device != dev || cache->n_ctx < 1 ||
+      cache->ld_v != round_up(cache->n_ctx, kKvTile) || (cache->ragged != 0 && cache->ragged != 1) ||
+      cache->filled != 1)
+    return SDM_ERR_CACHE_MISMATCH;
+  if (cache->k8 == nullptr || cache->v8t == nullptr || cache->scales == nullptr) return SDM_ERR_INVALID_ARG;
+  if (!aligned(cache->k8, 16) || !aligned(cache->v8t, 16) || !aligned(cache->scales, 16)) return SDM_ERR_INVALID_ARG;
+  if (!pinned_or_device(cache->k8, dev) || !pinned_or_device(cache->v8t, dev) || !on_device(cache->scales, dev))
+    return SDM_ERR_CACHE_MISMATCH;
+  if (c_h == nullptr || !aligned(c_h, 4)) return SDM_ERR_INVALID_ARG;
+  if (!on_device(c_h, dev)) return SDM_ERR_DEVICE_MISMATCH;
+  if (M == 0) return SDM_OK;
+  SDM_TRY(check_tensor(q, dev));
+  SDM_TRY(check_tensor(out, dev));
+  if (gate != nullptr) {
+    if (!aligned(gate, 2)) return SDM_ERR_INVALID_ARG;
+    if (!on_device(gate, dev)) return SDM_ERR_DEVICE_MISMATCH;
+  }
+  const int64_t N = cache->n_ctx;
+  const WsLayout w = ws_layout(SDM_OP_CACHED_ATTENTION_OFFLOAD, B, N, M, H, 1);
+  SDM_TRY(check_ws(ws, ws_bytes, w.total, dev));
+  cudaStream_t st = as_stream(stream);
+  cudaStream_t cs = copy_stream != nullptr ? as_stream(copy_stream) : st;
+  const bool overlap = cs != st;
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  const int64_t BH = (int64_t)B * H;
+  const int64_t L = split_keys_for(N);
+  const int64_t C = n_splits_for(N);
+  // events ordering the two streams: copies into a slot wait for the attention
+  // that last read it; an attention waits for its slot's copies
+  cudaEvent_t ev[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+  auto destroy = [&]() {
+    for (cudaEvent_t& e : ev)
+      if (e != nullptr) cudaEventDestroy(e);  // released once pending work completes
+  };
+  if (overlap) {
+    for (cudaEvent_t& e : ev)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+        cudaGetLastError();
+        destroy();
+        return SDM_ERR_CUDA;
+      }
+  }
+  cudaEvent_t start = ev[0], copied[2] = {ev[1], ev[2]}, used[2] = {ev[3], ev[4]};
+  sdm_status status = SDM_OK;
+  do {
+    if (overlap) {
+      // the slots may still be read by work enqueued on `stream` before this call
+      if (cudaEventRecord(start, st) != cudaSuccess || cudaStreamWaitEvent(cs, start, 0) != cudaSuccess) {
+        status = SDM_ERR_CUDA;
+        break;
+      }
+    }
+    // queries: scaled with the cache's n (n_b if ragged), quantised with its s_q
+    const float* meta = cache->scales + 3 * BH;
+    RowsDesc dq{reinterpret_cast<const __half*>(q), B, H, M};
+    QScale qs = make_qscale(N, c_h, gate);
+    if (cache->ragged) qs.lam_b = meta + B;
+    uint8_t* q8 = base + w.q8;
+    if (prepare_gate(qs, (int64_t)B * M * H, base, w, st) != cudaSuccess ||
+        launch_quantize_rows(dq, qs, M, cache->scales, q8, M, nullptr, 0, st) != cudaSuccess) {
+      status = SDM_ERR_CUDA;
+      break;
+    }
+    AttnArgs a;
+    a.B = B;
+    a.H = H;
+    a.T = M;
+    a.N = N;
+    a.ld_v = L;
+    a.kv_rows = L;
+    a.scales = cache->scales;
+    a.partial = true;
+    a.n_splits = 1;
+    a.split_keys = L;
+    a.out = reinterpret_cast<__half*>(out);
+    a.part_acc = reinterpret_cast<float*>(base + w.part_acc);
+    a.part_ml = reinterpret_cast<float*>(base + w.part_ml);
+    a.err = reinterpret_cast<uint32_t*>(base);
+    a.n_keys = cache->ragged ? reinterpret_cast<const int32_t*>(meta) : nullptr;
+    for (int64_t c = 0; c < C && status == SDM_OK; ++c) {
+      const int r = static_cast<int>(c & 1);
+      uint8_t* k_slot = base + w.stage + r * w.stage_bytes;
+      uint8_t* v_slot = k_slot + BH * L * kHeadDim;
+      const int64_t len = (N - c * L) < L ? (N - c * L) : L;      // keys of this chunk
+      const int64_t vlen = (cache->ld_v - c * L) < L ? (cache->ld_v - c * L) : L;  // with V's zero padding
+      if (overlap && c >= 2 && cudaStreamWaitEvent(cs, used[r], 0) != cudaSuccess) status = SDM_ERR_CUDA;
+      // K8 rows [cL, cL + len) of every (b, h); V8^T columns [cL, cL + vlen) of every (b, h, e)
+      if (status == SDM_OK &&
+          (cudaMemcpy2DAsync(k_slot, L * kHeadDim, cache->k8 + c * L * kHeadDim, N * kHeadDim, len * kHeadDim, BH,
+                             cudaMemcpyDefault, cs) != cudaSuccess ||
+           cudaMemcpy2DAsync(v_slot, L, cache->v8t + c * L, cache->ld_v, vlen, BH * kHeadDim, cudaMemcpyDefault,
+                             cs) != cudaSuccess))
+        status = SDM_ERR_CUDA;
+      if (status == SDM_OK && overlap &&
+          (cudaEventRecord(copied[r], cs) != cudaSuccess || cudaStreamWaitEvent(st, copied[r], 0) != cudaSuccess))
+        status = SDM_ERR_CUDA;
+      a.key_base = c * L;
+      a.split_base = c;
+      if (status == SDM_OK && launch_attention(q8, k_slot, v_slot, a, st) != cudaSuccess) status = SDM_ERR_CUDA;
+      if (status == SDM_OK && overlap && cudaEventRecord(used[r], st) != cudaSuccess) status = SDM_ERR_CUDA;
+    }
+    if (status != SDM_OK) break;
+    a.n_splits = C;
+    if (launch_splitkv_reduce(a, st) != cudaSuccess) status = SDM_ERR_CUDA;
+  } while (false);
+  if (status != SDM_OK) cudaGetLastError();
+  destroy();
+  return status;
+}
 
 sdm_status sdm_selftest_wait_timeout(void* ws, int64_t limit_cycles, void* stream) {
   if (ws == nullptr || !aligned(ws, 256)) return SDM_ERR_INVALID_ARG;

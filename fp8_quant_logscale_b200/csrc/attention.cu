@@ -98,6 +98,8 @@ struct KParams {
   uint32_t* err;
   const int32_t* n_keys;  // [B] keys per batch, or nullptr: N
   int32_t pad_rows;       // rows [n_b, N) are padding: written as zeros
+  int64_t key_base;       // global index of the K/V buffers' first key (a staged chunk), else 0
+  int64_t split_base;     // split index of this launch's first chunk in the partials, else 0
 };
 
 template <class S>
@@ -176,7 +178,7 @@ __global__ void __launch_bounds__(Cfg<kTiles>::kThreads, Cfg<kTiles>::kMinBlocks
   const int64_t bh = rest / p.n_splits;
   const int64_t row0 = pair * (kTiles * kQTile);
   const int64_t n_b = p.n_keys != nullptr ? (int64_t)__ldg(p.n_keys + bh / p.H) : p.N;  // this batch's keys
-  const int64_t kv_begin = p.partial ? split * p.split_keys : 0;
+  const int64_t kv_begin = p.partial ? p.key_base + split * p.split_keys : 0;  // global key index
   const int64_t kv_end = p.partial ? min(n_b, kv_begin + p.split_keys) : n_b;
   // no work: a key chunk past the batch's keys, or a CTA whose rows are all
   // padding context rows; the epilogue then writes neutral partials / zeros
@@ -233,7 +235,7 @@ __global__ void __launch_bounds__(Cfg<kTiles>::kThreads, Cfg<kTiles>::kMinBlocks
           raise_abort(s, p.err, kErrTimeoutEmpty);
           break;
         }
-        const int32_t key0 = static_cast<int32_t>(kv_begin + (int64_t)it * kKvTile);
+        const int32_t key0 = static_cast<int32_t>(kv_begin - p.key_base + (int64_t)it * kKvTile);  // in the buffer
         mbar_arrive_expect_tx(&s.k_full[st], kKBytes);
         tma_load_3d(s.k[st], &tm_k, &s.k_full[st], 0, key0, static_cast<int32_t>(bh));
         mbar_arrive_expect_tx(&s.v_full[st], kVLoadBytes);
@@ -483,7 +485,7 @@ __global__ void __launch_bounds__(Cfg<kTiles>::kThreads, Cfg<kTiles>::kMinBlocks
             dst[v] = zero ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(w[0], w[1], w[2], w[3]);
           }
         } else {
-          const int64_t prow = (split * p.BH + bh) * p.T + row;
+          const int64_t prow = ((split + p.split_base) * p.BH + bh) * p.T + row;
           float4* dst = reinterpret_cast<float4*>(p.part_acc + prow * kHeadDim);
 #pragma unroll
           for (int v = 0; v < 8; ++v)
@@ -507,7 +509,7 @@ __global__ void __launch_bounds__(Cfg<kTiles>::kThreads, Cfg<kTiles>::kMinBlocks
 #pragma unroll
           for (int v = 0; v < 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
         } else {
-          const int64_t prow = (split * p.BH + bh) * p.T + row;
+          const int64_t prow = ((split + p.split_base) * p.BH + bh) * p.T + row;
           float4* dst = reinterpret_cast<float4*>(p.part_acc + prow * kHeadDim);
 #pragma unroll
           for (int v = 0; v < 16; ++v) dst[v] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
@@ -624,10 +626,11 @@ cudaError_t launch_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CU
 cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8t, const AttnArgs& a,
                              cudaStream_t st) {
   const int64_t BH = (int64_t)a.B * a.H;
+  const int64_t kv_rows = a.kv_rows > 0 ? a.kv_rows : a.N;  // keys in the K8 buffer
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, q8, kHeadDim, a.T, BH, kHeadDim, a.T * kHeadDim, kHeadDim, kQTile,
                 CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !make_map(&tk, k8, kHeadDim, a.N, BH, kHeadDim, a.N * kHeadDim, kHeadDim, kKvTile,
+      !make_map(&tk, k8, kHeadDim, kv_rows, BH, kHeadDim, kv_rows * kHeadDim, kHeadDim, kKvTile,
                 CU_TENSOR_MAP_SWIZZLE_64B) ||
       !make_map(&tv, v8t, a.ld_v, kHeadDim, BH, a.ld_v, a.ld_v * kHeadDim, kKvTile, kHeadDim,
                 CU_TENSOR_MAP_SWIZZLE_128B))
@@ -647,6 +650,8 @@ cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t
   p.err = a.err;
   p.n_keys = a.n_keys;
   p.pad_rows = a.pad_rows ? 1 : 0;
+  p.key_base = a.key_base;
+  p.split_base = a.split_base;
   // at most 128 rows (small prediction batches): one query tile per CTA, two CTAs per SM
   if (a.T <= kQTile) return launch_kernel<1>(tq, tk, tv, p, BH, st);
   return launch_kernel<2>(tq, tk, tv, p, BH, st);

@@ -103,8 +103,14 @@ struct AttnArgs {
   float* part_acc;     // split: [S][B*H][T][64]
   float* part_ml;      // split: [S][B*H][T][2] (m2, l)
   uint32_t* err;       // device error word
-  const int32_t* n_keys;  // [B] keys per batch (ragged contexts), or nullptr: N for every batch
-  bool pad_rows;       // rows [n_keys[b], N) are padding context rows: written as zeros
+  const int32_t* n_keys = nullptr;  // [B] keys per batch (ragged contexts), or nullptr: N for every batch
+  bool pad_rows = false;  // rows [n_keys[b], N) are padding context rows: written as zeros
+  // A staged chunk of a cache held elsewhere: the K8 / V8^T buffers hold keys
+  // [key_base, key_base + kv_rows) of the N; the launch (partial, one split of
+  // split_keys keys) writes its partials at split index split_base.
+  int64_t kv_rows = 0;     // rows of the K8 buffer (0: N)
+  int64_t key_base = 0;
+  int64_t split_base = 0;
 };
 
 // Builds the tensor maps and launches the tcgen05 attention kernel.

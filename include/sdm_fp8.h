@@ -64,7 +64,8 @@ typedef enum {
   SDM_OP_QUANTIZE_CONTEXT = 0,
   SDM_OP_ICL_ATTENTION = 1,
   SDM_OP_CACHED_ATTENTION = 2,
-  SDM_OP_ICL_ATTENTION_F16 = 3
+  SDM_OP_ICL_ATTENTION_F16 = 3,
+  SDM_OP_CACHED_ATTENTION_OFFLOAD = 4
 } sdm_op;
 
 /* Keys per online-softmax block (blocks start at key 0, or at the chunk start
@@ -272,6 +273,26 @@ sdm_status sdm_icl_attention_f16_ragged(const void* q, const void* k, const void
                                         int64_t n_query, int32_t heads, int32_t head_dim, const int64_t* ctx_len,
                                         const float* c_h, const void* gate, void* out, void* ws, size_t ws_bytes,
                                         void* stream);
+
+/*
+ * Step 4 from a cache held off the device ("Cache chunking, CPU offloading
+ * ... are supported", "[FP8 3/4] ...", opening section).  Same result, bit
+ * for bit, as sdm_cached_attention on the same cache: the K8 / V8^T buffers
+ * (cache->k8, cache->v8t; page-locked host memory, or device memory) are
+ * streamed one split-KV chunk of sdm_split_keys(N) keys at a time into two
+ * staging slots of the workspace; chunk c's attention writes partial c and the
+ * fixed-order combine follows.  Only the scales block must be on the device.
+ * Copies run on `copy_stream` and overlap the attention of the previous chunk
+ * on `stream` (copy_stream NULL or equal to stream: one stream, no overlap);
+ * the call creates and releases its own events.  The cache must have been
+ * filled on the device (the caller copies k8 / v8t out; `filled` stays 1).
+ *   ws  >= sdm_workspace_size(SDM_OP_CACHED_ATTENTION_OFFLOAD, B, N, M, H, d, 0)
+ *       (holds 2 x B x H x 128 x sdm_split_keys(N) bytes of staging)
+ */
+sdm_status sdm_cached_attention_offload(const void* q, int32_t batch, int64_t n_query, int32_t heads,
+                                        int32_t head_dim, const sdm_fp8_cache* cache, const float* c_h,
+                                        const void* gate, void* out, void* ws, size_t ws_bytes, void* stream,
+                                        void* copy_stream);
 
 /*
  * Step 2 without a workspace.  This entry point has no counterpart in the
