@@ -160,3 +160,52 @@ def make_inputs(w: Workload, seed: int | None = None, n_ctx: int | None = None, 
         _normal_fill(qq, s, "queries")
         out["queries"] = qq.astype(np.float16)
     return out
+
+
+# --- ragged grouped-query prefill (a second workload, bf16, head dim 128) ---------
+
+@dataclasses.dataclass(frozen=True)
+class PrefillWorkload:
+    name: str
+    q_lens: tuple          # query tokens per sequence
+    kv_lens: tuple         # key/value tokens per sequence (the queries are the last q_len of them)
+    q_heads: int
+    kv_heads: int
+    head_dim: int = 128
+    causal: bool = True
+    seed: int = 0
+    description: str = ""
+
+
+PREFILL_WORKLOADS = {
+    "gqa4_prefill_b2": PrefillWorkload(
+        "gqa4_prefill_b2", (32, 64), (256, 1024), 16, 4, seed=11,
+        description="2 sequences, query lengths 32/64, key/value lengths 256/1024, 16 query heads sharing "
+                    "4 key/value heads, head dim 128, bf16 N(0,1); causal, queries aligned to the end"),
+}
+
+
+def bf16_bits(x32: np.ndarray) -> np.ndarray:
+    """float32 -> bf16 bit patterns, round to nearest even (input preparation only)."""
+    u = np.ascontiguousarray(x32, np.float32).view(np.uint32).astype(np.uint64)
+    r = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return r.astype(np.uint16)
+
+
+def make_prefill_inputs(w: PrefillWorkload, seed: int | None = None, q_lens=None, kv_lens=None) -> dict:
+    """Packed ragged inputs: q [sum q_len, Hq, d], k / v [sum kv_len, Hkv, d] as bf16 bits
+    (uint16), with host indptr arrays (int64, B + 1 entries)."""
+    s = w.seed if seed is None else seed
+    q_lens = tuple(w.q_lens if q_lens is None else q_lens)
+    kv_lens = tuple(w.kv_lens if kv_lens is None else kv_lens)
+    qo = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int64)
+    kvo = np.concatenate([[0], np.cumsum(kv_lens)]).astype(np.int64)
+    out = {}
+    for name, rows, heads in (("q", int(qo[-1]), w.q_heads), ("k", int(kvo[-1]), w.kv_heads),
+                              ("v", int(kvo[-1]), w.kv_heads)):
+        x = np.empty((rows, heads, w.head_dim), np.float32)
+        _normal_fill(x, s, name)
+        out[name] = bf16_bits(x)
+    out.update(qo_indptr=qo, kv_indptr=kvo, q_lens=q_lens, kv_lens=kv_lens, q_heads=w.q_heads,
+               kv_heads=w.kv_heads, head_dim=w.head_dim, causal=w.causal, workload=w)
+    return out

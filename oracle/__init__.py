@@ -217,8 +217,9 @@ def attention_exact(q, k, v, rows=None):
         rows = np.arange(T, dtype=np.int64)
     rows = np.ascontiguousarray(rows, np.int64)
     out = np.empty((B, rows.size, H, d), np.float64)
-    lib().orc_attention_exact(_ptr(_bits16(q)), _ptr(_bits16(k)), _ptr(_bits16(v)),
-                              B, H, T, N, d, _ptr(rows), rows.size, _ptr(out))
+    # keep the (possibly copied) contiguous inputs alive for the duration of the call
+    qb, kb, vb = _bits16(q), _bits16(k), _bits16(v)
+    lib().orc_attention_exact(_ptr(qb), _ptr(kb), _ptr(vb), B, H, T, N, d, _ptr(rows), rows.size, _ptr(out))
     return out
 
 
@@ -295,4 +296,46 @@ def attention_exact_ragged(q, k, v, ctx_len, rows=None):
         if sel.size:
             out[b, sel] = attention_exact(np.ascontiguousarray(q[b:b + 1]), np.ascontiguousarray(k[b:b + 1, :n]),
                                           np.ascontiguousarray(v[b:b + 1, :n]), rows=rows[sel])[0]
+    return out
+
+
+# --- ragged grouped-query prefill (bf16 in, exact softmax) ----------------------
+
+def bf16_decode(bits) -> np.ndarray:
+    """bf16 bit patterns -> float64 (a bf16 value is the top 16 bits of a float32)."""
+    b = np.ascontiguousarray(bits, np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def gqa_prefill(q, k, v, qo_indptr, kv_indptr, q_heads: int, kv_heads: int, causal: bool = True):
+    """Attention of a packed ragged batch with grouped-query heads, in double precision.
+
+    Sequence b owns query tokens [qo[b], qo[b+1]) and key/value tokens [kv[b], kv[b+1]);
+    query head h reads key/value head h // (q_heads / kv_heads); scores are scaled by
+    1/sqrt(d).  Causal (the queries are the last q_len of the kv_len tokens): query i
+    attends keys j <= kv_len - q_len + i.  q [Tq, Hq, d], k/v [Tkv, Hkv, d] as bf16 bits.
+    Returns out [Tq, Hq, d] float64.
+    """
+    qd, kd, vd = bf16_decode(q), bf16_decode(k), bf16_decode(v)
+    Tq, Hq, d = qd.shape
+    assert Hq == q_heads and kd.shape[1] == kv_heads and q_heads % kv_heads == 0
+    G = q_heads // kv_heads
+    out = np.zeros((Tq, Hq, d))
+    for b in range(len(qo_indptr) - 1):
+        q0, q1 = int(qo_indptr[b]), int(qo_indptr[b + 1])
+        k0, k1 = int(kv_indptr[b]), int(kv_indptr[b + 1])
+        nq, nk = q1 - q0, k1 - k0
+        if nq == 0:
+            continue
+        allowed = np.ones((nq, nk), bool)
+        if causal:
+            assert nk >= nq, "causal prefill needs kv_len >= q_len"
+            allowed = np.arange(nk)[None, :] <= (nk - nq + np.arange(nq))[:, None]
+        for h in range(Hq):
+            g = h // G
+            s = (qd[q0:q1, h] @ kd[k0:k1, g].T) / np.sqrt(d)
+            s = np.where(allowed, s, -np.inf)
+            s = s - s.max(axis=1, keepdims=True)
+            p = np.exp(s)
+            out[q0:q1, h] = (p / p.sum(axis=1, keepdims=True)) @ vd[k0:k1, g]
     return out
