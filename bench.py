@@ -487,6 +487,76 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_prefill(args):
+    """The ragged grouped-query prefill workload (bf16, head dim 128) through sdm_gqa_prefill: one
+    launch timed alone (median of K after W), and 100 back-to-back launches between two events, the
+    pages' per-sample protocol (they report 37.04 us, FlashInfer 21.93 us, on an H20)."""
+    import torch
+
+    import fp8_quant_logscale_b200 as sdm
+    from fp8_quant_logscale_b200 import binding
+    from fp8_quant_logscale_b200.workloads import PREFILL_WORKLOADS, make_prefill_inputs
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    w = PREFILL_WORKLOADS["gqa4_prefill_b2"]
+    inp = make_prefill_inputs(w)
+    dev = lambda x: torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
+    q, k, v = dev(inp["q"]), dev(inp["k"]), dev(inp["v"])
+    out = torch.empty_like(q)
+    qo, kvo = inp["qo_indptr"], inp["kv_indptr"]
+    ws = sdm.new_workspace(binding.gqa_prefill_workspace_size(qo, kvo, w.q_heads, w.kv_heads, w.causal), device)
+    visible = sum((kl - ql) * ql + ql * (ql + 1) // 2 for ql, kl in zip(w.q_lens, w.kv_lens))
+    flops = 4.0 * w.head_dim * w.q_heads * visible
+    call = lambda: sdm.gqa_prefill(q, k, v, qo, kvo, causal=w.causal, out=out, ws=ws)
+    stream = torch.cuda.current_stream(device)
+    single = []
+    for i in range(args.warmup + args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        call()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        if i >= args.warmup:
+            single.append(a.elapsed_time(b) * 1e3)
+    batch = []
+    for i in range(args.warmup + args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(100):
+            call()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        if i >= args.warmup:
+            batch.append(a.elapsed_time(b) * 1e3 / 100)
+    # device time: one call captured in a CUDA graph, replayed 100 times between two events
+    side = torch.cuda.Stream(device)
+    with torch.cuda.stream(side):
+        call()
+        torch.cuda.synchronize(device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            call()
+    graph = []
+    for i in range(args.warmup + args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(100):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        if i >= args.warmup:
+            graph.append(a.elapsed_time(b) * 1e3 / 100)
+    peaks = measured_peaks() or {"bf16_tflops": 1590.0}
+    us = statistics.median(graph)
+    print(json.dumps({"step": "a9 ragged GQA4 prefill, bf16 (sdm_gqa_prefill)", "workload": w.name,
+                      "us_per_launch_graph": us, "us_per_launch_eager_100": statistics.median(batch),
+                      "us_single_launch_eager": statistics.median(single),
+                      "flops": flops, "tflops": flops / (us * 1e-6) / 1e12,
+                      "frac_bf16": flops / (us * 1e-6) / 1e12 / peaks["bf16_tflops"],
+                      "pages": "37.04 us (oxide), 21.93 us (FlashInfer), H20, eager"}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -499,6 +569,7 @@ def main(argv=None):
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--per-kernel", action="store_true",
                     help="time each step of the path alone (one JSON line per step) instead of the benchmark step")
+    ap.add_argument("--prefill", action="store_true", help="time the ragged grouped-query prefill workload")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per attention launch from an ncu capture of the current kernel")
     args = ap.parse_args(argv)
@@ -506,6 +577,8 @@ def main(argv=None):
         run_reference(args)
     elif args.per_kernel:
         run_per_kernel(args)
+    elif args.prefill:
+        run_prefill(args)
     else:
         run_ours(args)
 

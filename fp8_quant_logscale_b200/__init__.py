@@ -8,10 +8,10 @@ cached prediction over a resident FP8 K/V cache; plus the normal-precision
 short contexts.
 """
 from .binding import (FP8Cache, OffloadedFP8Cache, SdmError, cached_attention, cached_attention_offload,
-                      fp8_attention, fp8_eligible, fp8_quantize_context, icl_attention, icl_attention_f16, icl_layer,
-                      lib, new_workspace, qscale_fused, sync_status, workspace_size)
+                      fp8_attention, fp8_eligible, fp8_quantize_context, gqa_prefill, icl_attention, icl_attention_f16,
+                      icl_layer, lib, new_workspace, qscale_fused, sync_status, workspace_size)
 
 __all__ = ["FP8Cache", "OffloadedFP8Cache", "SdmError", "cached_attention", "cached_attention_offload",
-           "fp8_attention", "fp8_eligible", "fp8_quantize_context",
+           "fp8_attention", "fp8_eligible", "fp8_quantize_context", "gqa_prefill",
            "icl_attention", "icl_attention_f16", "icl_layer", "lib", "new_workspace", "qscale_fused", "sync_status",
            "workspace_size"]

@@ -28,7 +28,8 @@ HEAD_DIM = 64
 EXPORTS = ("sdm_status_string", "sdm_version", "sdm_split_keys", "sdm_cache_layout", "sdm_workspace_size", "sdm_qscale_fused",
            "sdm_fp8_quantize_context", "sdm_fp8_quantize_context_noalloc", "sdm_fp8_attention", "sdm_icl_attention",
            "sdm_cached_attention", "sdm_fp8_eligible", "sdm_icl_attention_f16", "sdm_icl_attention_ragged",
-           "sdm_icl_attention_f16_ragged", "sdm_cached_attention_offload", "sdm_sync_status",
+           "sdm_icl_attention_f16_ragged", "sdm_cached_attention_offload", "sdm_gqa_prefill",
+           "sdm_gqa_prefill_workspace_size", "sdm_sync_status",
            "sdm_selftest_wait_timeout")
 NOALLOC_MAX_BATCH_HEADS = 4096
 
@@ -94,6 +95,10 @@ def lib() -> ctypes.CDLL:
         L.sdm_cached_attention_offload.restype = ctypes.c_int
         L.sdm_cached_attention_offload.argtypes = [_P, _I32, _I64, _I32, _I32, ctypes.POINTER(CacheStruct), _P, _P,
                                                    _P, _P, _SZ, _P, _P]
+        L.sdm_gqa_prefill.restype = ctypes.c_int
+        L.sdm_gqa_prefill.argtypes = [_P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P, _P, _SZ, _P]
+        L.sdm_gqa_prefill_workspace_size.restype = _SZ
+        L.sdm_gqa_prefill_workspace_size.argtypes = [_P, _P, _I32, _I32, _I32, _I32, _I32]
         L.sdm_fp8_eligible.restype = _I32
         L.sdm_fp8_eligible.argtypes = [_I64, _I32]
         L.sdm_icl_attention_f16.restype = ctypes.c_int
@@ -445,3 +450,33 @@ def cached_attention_offload(q: torch.Tensor, cache: OffloadedFP8Cache, c_h: tor
                                                   ctypes.c_void_p(copy_stream.cuda_stream)),
                "sdm_cached_attention_offload")
     return out
+
+
+def gqa_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, qo_indptr, kv_indptr, causal: bool = True,
+                out: torch.Tensor | None = None, ws: torch.Tensor | None = None) -> torch.Tensor:
+    """Ragged grouped-query prefill: q [total_q, Hq, 128], k / v [total_kv, Hkv, 128] bf16, host indptr
+    sequences of batch + 1 offsets -> out [total_q, Hq, 128] bf16."""
+    _want(q, torch.bfloat16, "q", 3)
+    _want(k, torch.bfloat16, "k", 3)
+    _want(v, torch.bfloat16, "v", 3)
+    qo = (ctypes.c_int64 * len(qo_indptr))(*[int(x) for x in qo_indptr])
+    kvo = (ctypes.c_int64 * len(kv_indptr))(*[int(x) for x in kv_indptr])
+    if len(qo_indptr) != len(kv_indptr):
+        raise ValueError("qo_indptr and kv_indptr must have the same length")
+    dev = q.device
+    out = torch.empty_like(q) if out is None else out
+    if ws is None:
+        ws = new_workspace(gqa_prefill_workspace_size(qo_indptr, kv_indptr, q.shape[1], k.shape[1], causal), dev)
+    with torch.cuda.device(dev):
+        _check(lib().sdm_gqa_prefill(_ptr(q), _ptr(k), _ptr(v), qo, kvo, len(qo_indptr) - 1, q.shape[1], k.shape[1],
+                                     q.shape[2], 1 if causal else 0, _ptr(out), _ptr(ws), ws.numel(), _stream(dev)),
+               "sdm_gqa_prefill")
+    return out
+
+
+def gqa_prefill_workspace_size(qo_indptr, kv_indptr, q_heads: int, kv_heads: int, causal: bool = True) -> int:
+    """Workspace bytes sdm_gqa_prefill needs for this batch (0 for an invalid batch)."""
+    qo = (ctypes.c_int64 * len(qo_indptr))(*[int(x) for x in qo_indptr])
+    kvo = (ctypes.c_int64 * len(kv_indptr))(*[int(x) for x in kv_indptr])
+    return int(lib().sdm_gqa_prefill_workspace_size(qo, kvo, len(qo_indptr) - 1, q_heads, kv_heads, 128,
+                                                    1 if causal else 0))

@@ -14,7 +14,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsdm_fp8.so")
-SOURCES = ["api.cu", "quant.cu", "attention.cu", "attention_f16.cu"]
+SOURCES = ["api.cu", "quant.cu", "attention.cu", "attention_f16.cu", "prefill.cu"]
 HEADERS = ["kernels.cuh", "ptx.cuh", "exp2_poly.cuh", "softmax.cuh", os.path.join("..", "..", "include", "sdm_fp8.h")]
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <mutex>
+#include <vector>
 
 #include "../../include/sdm_fp8.h"
 #include "kernels.cuh"
@@ -712,6 +713,61 @@ sdm_status sdm_cached_attention_offload(const void* q, int32_t B, int64_t M, int
   if (status != SDM_OK) cudaGetLastError();
   destroy();
   return status;
+}
+
+// Host-side checks of a prefill batch; fills seqs on success.
+static sdm_status prefill_batch(const int64_t* qo_indptr, const int64_t* kv_indptr, int32_t batch, int32_t q_heads,
+                                int32_t kv_heads, int32_t head_dim, int32_t causal, std::vector<PrefillSeq>& seqs) {
+  if (batch < 0 || qo_indptr == nullptr || kv_indptr == nullptr) return SDM_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SDM_ERR_INVALID_ARG;
+  if (head_dim != 128) return SDM_ERR_UNSUPPORTED;
+  if (q_heads < 1 || kv_heads < 1 || q_heads % kv_heads != 0) return SDM_ERR_INVALID_ARG;
+  const int32_t G = q_heads / kv_heads;
+  if (G > 16 || (G & (G - 1)) != 0 || q_heads > 256 || kv_heads > 256) return SDM_ERR_UNSUPPORTED;
+  for (const int64_t* ip : {qo_indptr, kv_indptr}) {  // host arrays of batch + 1 offsets
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, ip) == cudaSuccess) {
+      if (at.type == cudaMemoryTypeDevice) return SDM_ERR_INVALID_ARG;
+    } else {
+      cudaGetLastError();
+    }
+  }
+  if (qo_indptr[0] != 0 || kv_indptr[0] != 0) return SDM_ERR_INVALID_ARG;
+  seqs.resize(static_cast<size_t>(batch));
+  for (int32_t b = 0; b < batch; ++b) {
+    const int64_t ql = qo_indptr[b + 1] - qo_indptr[b], kl = kv_indptr[b + 1] - kv_indptr[b];
+    if (ql < 0 || kl < 0 || (ql > 0 && kl < 1) || (causal && kl < ql)) return SDM_ERR_INVALID_ARG;
+    seqs[b] = PrefillSeq{qo_indptr[b], ql, kv_indptr[b], kl};
+  }
+  // TMA coordinates and the kernel's offsets are 32-bit
+  if (qo_indptr[batch] > ((int64_t)1 << 30) || kv_indptr[batch] > ((int64_t)1 << 30)) return SDM_ERR_UNSUPPORTED;
+  return SDM_OK;
+}
+
+size_t sdm_gqa_prefill_workspace_size(const int64_t* qo_indptr, const int64_t* kv_indptr, int32_t batch,
+                                      int32_t q_heads, int32_t kv_heads, int32_t head_dim, int32_t causal) {
+  std::vector<PrefillSeq> seqs;
+  if (prefill_batch(qo_indptr, kv_indptr, batch, q_heads, kv_heads, head_dim, causal, seqs) != SDM_OK) return 0;
+  return gqa_prefill_ws_bytes(seqs.data(), batch, q_heads, kv_heads, causal);
+}
+
+sdm_status sdm_gqa_prefill(const void* q, const void* k, const void* v, const int64_t* qo_indptr,
+                           const int64_t* kv_indptr, int32_t batch, int32_t q_heads, int32_t kv_heads,
+                           int32_t head_dim, int32_t causal, void* out, void* ws, size_t ws_bytes, void* stream) {
+  std::vector<PrefillSeq> seqs;
+  SDM_TRY(prefill_batch(qo_indptr, kv_indptr, batch, q_heads, kv_heads, head_dim, causal, seqs));
+  const int64_t total_q = qo_indptr[batch], total_kv = kv_indptr[batch];
+  if (total_q == 0) return SDM_OK;
+  const int dev = current_device();
+  if (dev < 0) return SDM_ERR_CUDA;
+  SDM_TRY(check_tensor(q, dev));
+  SDM_TRY(check_tensor(k, dev));
+  SDM_TRY(check_tensor(v, dev));
+  SDM_TRY(check_tensor(out, dev));
+  SDM_TRY(check_ws(ws, ws_bytes, gqa_prefill_ws_bytes(seqs.data(), batch, q_heads, kv_heads, causal), dev));
+  SDM_CUDA(launch_gqa_prefill(q, k, v, total_q, total_kv, seqs.data(), batch, q_heads, kv_heads, causal, out,
+                              reinterpret_cast<uint8_t*>(ws), as_stream(stream)));
+  return SDM_OK;
 }
 
 sdm_status sdm_selftest_wait_timeout(void* ws, int64_t limit_cycles, void* stream) {

@@ -89,6 +89,23 @@ cudaError_t launch_attention_f16(const __half* q_scaled, const __half* k, const 
                                  int64_t N, int32_t H, int64_t ld_v, const int32_t* n_keys, __half* out,
                                  uint32_t* err, cudaStream_t st);
 
+// Ragged grouped-query prefill (bf16, head dim 128): one sequence's token ranges
+// in the packed q and k/v tensors.  Sequences are launched 64 at a time.
+constexpr int kPrefillMaxSeqs = 64;
+struct PrefillSeq {
+  int64_t q_off, q_len, kv_off, kv_len;
+};
+// out [total_q][q_heads][128] = attention of q [total_q][q_heads][128] to k, v
+// [total_kv][kv_heads][128] (bf16), query head h reading key/value head
+// h / (q_heads / kv_heads); causal: the queries are the last q_len keys.
+// ws: the error word, then per-launch tickets (zero between launches; the
+// kernel returns them to zero) and the partials of split key ranges.
+cudaError_t launch_gqa_prefill(const void* q, const void* k, const void* v, int64_t total_q, int64_t total_kv,
+                               const PrefillSeq* seqs, int32_t n_seqs, int32_t q_heads, int32_t kv_heads,
+                               int32_t causal, void* out, uint8_t* ws, cudaStream_t st);
+size_t gqa_prefill_ws_bytes(const PrefillSeq* seqs, int32_t n_seqs, int32_t q_heads, int32_t kv_heads,
+                            int32_t causal);
+
 // ---------------------------------------------------------------- attention
 struct AttnArgs {
   int32_t B, H;

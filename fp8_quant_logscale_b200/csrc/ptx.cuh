@@ -126,6 +126,15 @@ __device__ __forceinline__ uint64_t smem_desc_kmajor(uint32_t saddr, uint32_t sb
 constexpr uint32_t kSwizzle128B = 2;
 constexpr uint32_t kSwizzle64B = 4;
 
+// Shared-memory matrix descriptor, MN-major operand with the 128-byte swizzle:
+// each 128-byte row holds 128 bytes of the M/N dimension for one k; 8 rows
+// (k, k+1, ..) form a 1 KB swizzle atom; `lbo_bytes` is the distance between
+// consecutive 128-byte M/N atoms, `sbo_bytes` between consecutive 8-row k groups.
+__device__ __forceinline__ uint64_t smem_desc_mnmajor_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | ((uint64_t)1u << 46) | ((uint64_t)kSwizzle128B << 61);
+}
+
 // Instruction descriptor for kind::f8f6f4, E4M3 x E4M3 -> F32, both operands K-major.
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
   return (1u << 4)                      // D format: F32
@@ -153,6 +162,15 @@ __device__ __forceinline__ void mma_e4m3_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+// Instruction descriptor for kind::f16, BF16 x BF16 -> F32; A K-major, B K-major
+// (b_mn_major = false) or MN-major (true).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
+  return (1u << 4)                      // D format: F32
+         | (1u << 7) | (1u << 10)       // A, B format: BF16
+         | ((b_mn_major ? 1u : 0u) << 16)
+         | ((uint32_t)(N >> 3) << 17)   // N / 8
+         | ((uint32_t)(M >> 4) << 24);  // M / 16
 }
 // Instruction descriptor for kind::f16, F16 x F16 -> F32, both operands K-major.
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
@@ -280,6 +298,12 @@ __device__ __forceinline__ void sub2(float& d0, float& d1, float a0, float a1, f
 __device__ __forceinline__ uint32_t f16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// Two floats -> bf16x2 (round to nearest even), `lo` in bits 0..15.
+__device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
 // 2^x, hardware approximation (flush-to-zero).

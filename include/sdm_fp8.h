@@ -295,6 +295,35 @@ sdm_status sdm_cached_attention_offload(const void* q, int32_t batch, int64_t n_
                                         void* copy_stream);
 
 /*
+ * Ragged grouped-query prefill, a second workload beside the ICL layer
+ * ("Pipeline long ragged GQA4 KV loads", oxide-infer PR #114, performance
+ * contract: 2 sequences, query lengths 32/64, key/value lengths 256/1024, 16
+ * query heads, 4 key/value heads, head dim 128, bf16).  Sequence b owns query
+ * tokens [qo_indptr[b], qo_indptr[b+1]) and key/value tokens [kv_indptr[b],
+ * kv_indptr[b+1]); query head h reads key/value head h / (q_heads / kv_heads);
+ * out = softmax(q k^T / sqrt(128)) v with fp32 softmax and accumulation.
+ * causal = 1: the queries are the last q_len of the kv_len tokens, query i
+ * sees keys j <= kv_len - q_len + i (needs kv_len >= q_len); causal = 0: every
+ * key of the sequence.
+ *   q    [total_q][q_heads][128] bf16;  k, v [total_kv][kv_heads][128] bf16
+ *   qo_indptr, kv_indptr  HOST arrays of batch + 1 int64 offsets, starting at 0
+ *   out  [total_q][q_heads][128] bf16
+ *   q_heads / kv_heads in {1, 2, 4, 8, 16}; head_dim 128 (else SDM_ERR_UNSUPPORTED)
+ *   ws   >= sdm_gqa_prefill_workspace_size(...) bytes, all zero before its first
+ *        use: the error word, one ticket per (query tile, key/value head) --
+ *        the kernel returns them to zero -- and the partial results of the
+ *        256-key chunks a query tile's keys are split into (the last CTA of a
+ *        tile to finish combines them in chunk order).
+ * This entry point has no counterpart on the pages that define the ICL layer.
+ */
+size_t sdm_gqa_prefill_workspace_size(const int64_t* qo_indptr, const int64_t* kv_indptr, int32_t batch,
+                                      int32_t q_heads, int32_t kv_heads, int32_t head_dim, int32_t causal);
+
+sdm_status sdm_gqa_prefill(const void* q, const void* k, const void* v, const int64_t* qo_indptr,
+                           const int64_t* kv_indptr, int32_t batch, int32_t q_heads, int32_t kv_heads,
+                           int32_t head_dim, int32_t causal, void* out, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Step 2 without a workspace.  This entry point has no counterpart in the
  * pages: it exists for callers that cannot allocate device memory for the
  * library -- code that must not call cudaMalloc on its path (cudaMalloc can

@@ -119,3 +119,22 @@ def test_ragged_argument_errors(L):
     assert g(None, None, None, 2, 100, 5, 4, 64, lens(-3, 7), None, None, None, None, 0, None) == 1
     if not torch.cuda.is_available():  # valid lengths get past the host checks to the device query
         assert f(None, None, None, 2, 100, 5, 4, 64, lens(100, 1), None, None, None, None, None, 0, None) == 7
+
+
+def test_prefill_argument_errors(L):
+    import ctypes as C
+    ip = lambda *x: (C.c_int64 * len(x))(*x)
+    f = L.sdm_gqa_prefill
+    assert f(None, None, None, None, None, 1, 16, 4, 128, 1, None, None, 0, None) == 1      # no indptr
+    assert f(None, None, None, ip(0, 5), ip(0, 10), 1, 16, 4, 64, 1, None, None, 0, None) == 2   # head dim
+    assert f(None, None, None, ip(0, 5), ip(0, 10), 1, 16, 3, 128, 1, None, None, 0, None) == 1  # 16 % 3
+    assert f(None, None, None, ip(0, 5), ip(0, 10), 1, 64, 2, 128, 1, None, None, 0, None) == 2  # group 32
+    assert f(None, None, None, ip(0, 5), ip(0, 4), 1, 16, 4, 128, 1, None, None, 0, None) == 1   # kv < q, causal
+    assert f(None, None, None, ip(0, 5), ip(0, 0), 1, 16, 4, 128, 0, None, None, 0, None) == 1   # no keys
+    assert f(None, None, None, ip(1, 5), ip(0, 10), 1, 16, 4, 128, 1, None, None, 0, None) == 1  # offsets from 0
+    assert f(None, None, None, ip(0, 0), ip(0, 0), 1, 16, 4, 128, 1, None, None, 0, None) == 0   # nothing to do
+    # error word + tickets + partials of the 2048-key chunks: q 64 tokens in 2 tiles, 5000 keys -> 6 chunks
+    need = binding.gqa_prefill_workspace_size([0, 64], [0, 5000], 16, 4)
+    assert need >= 256 + 2 * 4 * 4 + 6 * 4 * 128 * (2 + 128) * 4
+    assert binding.gqa_prefill_workspace_size([0, 64], [0, 10], 16, 4) == 0          # kv < q, causal
+    assert binding.gqa_prefill_workspace_size([0, 64], [0, 10], 16, 4, causal=False) > 0
