@@ -98,8 +98,8 @@ struct PrefillSeq {
 // out [total_q][q_heads][128] = attention of q [total_q][q_heads][128] to k, v
 // [total_kv][kv_heads][128] (bf16), query head h reading key/value head
 // h / (q_heads / kv_heads); causal: the queries are the last q_len keys.
-// ws: the error word, then per-launch tickets (zero between launches; the
-// kernel returns them to zero) and the partials of split key ranges.
+// ws: the error word.  Each query tile is one cluster of 4 CTAs, each with a
+// quarter of the tile's keys; the cluster combines them in shared memory.
 cudaError_t launch_gqa_prefill(const void* q, const void* k, const void* v, int64_t total_q, int64_t total_kv,
                                const PrefillSeq* seqs, int32_t n_seqs, int32_t q_heads, int32_t kv_heads,
                                int32_t causal, void* out, uint8_t* ws, cudaStream_t st);

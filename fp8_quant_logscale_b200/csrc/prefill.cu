@@ -20,8 +20,6 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
-#include <vector>
-
 #include "kernels.cuh"
 #include "ptx.cuh"
 #include "softmax.cuh"
@@ -54,17 +52,17 @@ struct __align__(1024) SmemP {
   uint32_t last;  // this CTA is the last of its query tile's key chunks to finish
 };
 
+constexpr int kClusterP = 4;  // CTAs per query tile, each with a quarter of its keys
+constexpr int kStashLd = kDP + 4;  // floats per row of the shared-memory partials (padded)
+static_assert(kClusterP * 32 * kStashLd * 4 <= kStagesP * 2 * kHalfBytesP, "partials fit in the K stages");
+
 struct PrefillParams {
-  int32_t n_seqs, q_heads, kv_heads, group, tokens_per_tile, causal, split_keys;
+  int32_t n_seqs, q_heads, kv_heads, group, tokens_per_tile, causal;
   int32_t q_off[kPrefillMaxSeqs], q_len[kPrefillMaxSeqs], kv_off[kPrefillMaxSeqs], kv_len[kPrefillMaxSeqs];
   int32_t tile_start[kPrefillMaxSeqs + 1];  // prefix sum of query tiles over the sequences
-  int32_t item_start[kPrefillMaxSeqs + 1];  // prefix sum of (query tile, key chunk) work items
   float c2;                                 // log2(e) / sqrt(128)
   __nv_bfloat16* out;                       // [total_q][Hq][128]
   uint32_t* err;
-  uint32_t* tickets;                        // [tiles][kv_heads], zero between launches
-  float* part_ml;                           // [items][kv_heads][128][2]: m2, l
-  float* part_acc;                          // [items][kv_heads][128][128]
 };
 
 __device__ __forceinline__ void raise_abort_p(SmemP& s, uint32_t* err, uint32_t code) {
@@ -115,7 +113,7 @@ __device__ __forceinline__ void p_chunk_bf16(const uint32_t (&r)[32], uint32_t (
   }
 }
 
-__global__ void __launch_bounds__(kThreadsP, 1)
+__global__ void __cluster_dims__(kClusterP, 1, 1) __launch_bounds__(kThreadsP, 1)
     gqa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ PrefillParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -124,29 +122,21 @@ __global__ void __launch_bounds__(kThreadsP, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- which sequence, key/value head, query tile and key chunk
+  // ---- which sequence, key/value head and query tile; this CTA's share of the keys
+  const int rank = static_cast<int>(cluster_ctarank());       // 0..3 within the cluster
+  const int tile = static_cast<int>(blockIdx.x) / kClusterP;  // query tile over all sequences
   int b = 0;
-  while (b + 1 < p.n_seqs && p.item_start[b + 1] <= static_cast<int>(blockIdx.x)) ++b;
+  while (b + 1 < p.n_seqs && p.tile_start[b + 1] <= tile) ++b;
   const int kvh = blockIdx.y;
-  const int G = p.group, tpt = p.tokens_per_tile, L = p.split_keys;
+  const int G = p.group, tpt = p.tokens_per_tile;
   const int q_len = p.q_len[b], kv_len = p.kv_len[b];
-  // keys the rows of query tile t see: the causal limit of its last token
-  auto tile_keys = [&](int t) {
-    const int te = (t + 1) * tpt < q_len ? (t + 1) * tpt : q_len;
-    return p.causal ? kv_len - q_len + te : kv_len;
-  };
-  int qt = 0, chunk = static_cast<int>(blockIdx.x) - p.item_start[b], item0 = p.item_start[b];
-  while (true) {  // walk the tiles of sequence b to this item's (tile, chunk)
-    const int nc = (tile_keys(qt) + L - 1) / L;
-    if (chunk < nc) break;
-    chunk -= nc;
-    item0 += nc;
-    ++qt;
-  }
-  const int n_chunks = (tile_keys(qt) + L - 1) / L;
-  const int tok0 = qt * tpt;
-  const int kv_lo = chunk * L;
-  const int kv_hi = kv_lo + L < tile_keys(qt) ? kv_lo + L : tile_keys(qt);
+  const int tok0 = (tile - p.tile_start[b]) * tpt;
+  const int tok_end = tok0 + tpt < q_len ? tok0 + tpt : q_len;
+  const int n_keys = p.causal ? kv_len - q_len + tok_end : kv_len;  // keys any row of the tile sees
+  // the cluster's CTAs take consecutive runs of whole 128-key tiles
+  const int per = ((n_keys + kKvTile - 1) / kKvTile + kClusterP - 1) / kClusterP * kKvTile;
+  const int kv_lo = rank * per < n_keys ? rank * per : n_keys;
+  const int kv_hi = kv_lo + per < n_keys ? kv_lo + per : n_keys;
   const int n_tiles = (kv_hi - kv_lo + kKvTile - 1) / kKvTile;
 
   if (threadIdx.x == 0) {
@@ -172,6 +162,9 @@ __global__ void __launch_bounds__(kThreadsP, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
+  // what the softmax hands to the cluster's combine (one row per softmax thread)
+  bool have_share = false;  // this CTA's keys were attended (and no wait gave up)
+  float share_m2 = -INFINITY, share_l = 0.0f;
 
   if (warp == kProducerWarpP) {
     // ================================================================ TMA producer
@@ -371,111 +364,103 @@ __global__ void __launch_bounds__(kThreadsP, 1)
       if (!ok && lane == 0) raise_abort_p(s, p.err, kErrTimeoutO);
     }
     if (ok && n_tiles > 0) {
-      tc_fence_after();
-      const float lf = ((l[0] + l[1]) + (l[2] + l[3])) + ((l[4] + l[5]) + (l[6] + l[7]));
-      if (n_chunks == 1) {
-        // one reciprocal per row: x * RN(1/l) is within 1.5 fp32 ulp of x / l, far
-        // below the bf16 rounding that follows
-        const float rl = __frcp_rn(lf);
-        __nv_bfloat16* dst = p.out + ((int64_t)(p.q_off[b] + tok) * p.q_heads + kvh * G + r % G) * kDP;
-#pragma unroll
-        for (int c = 0; c < kDP / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld_32x32b_x32(t_o + 32 * c, o);
-          tmem_ld_wait();
-          if (valid) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint32_t w[4];
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                w[k] = bf16x2(__fmul_rn(__uint_as_float(o[8 * v + 2 * k]), rl),
-                              __fmul_rn(__uint_as_float(o[8 * v + 2 * k + 1]), rl));
-              d4[v] = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-          }
-        }
-      } else {
-        // one chunk of the keys: the unnormalised O, m2 and l for the combine
-        const int64_t prow = ((int64_t)(item0 + chunk) * p.kv_heads + kvh) * kQTile + r;
-        float4* acc = reinterpret_cast<float4*>(p.part_acc + prow * kDP);
-#pragma unroll
-        for (int c = 0; c < kDP / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld_32x32b_x32(t_o + 32 * c, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            acc[8 * c + v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
-                                         __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
-        }
-        reinterpret_cast<float2*>(p.part_ml)[prow] = make_float2(m2, lf);
-      }
+      have_share = true;
+      share_m2 = m2;
+      share_l = ((l[0] + l[1]) + (l[2] + l[3])) + ((l[4] + l[5]) + (l[6] + l[7]));
     }
   }
 
+  // ---- every CTA of the cluster is done with its keys (its K stages are free):
+  // the unnormalised O, m2 and l of row r go straight into the shared memory of
+  // the cluster CTA that finishes row r (rank r / 32), into the slot of this
+  // CTA's rank -- remote stores, no round trip -- so that after the next barrier
+  // every combine reads local memory.  Slots live in the K stages; rows padded
+  // to 132 floats so that a warp's 32 rows fall in different banks.
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp < 4) {
+    tc_fence_after();
+    const int r = 32 * warp + lane;
+    const uint32_t owner = static_cast<uint32_t>(r >> 5);
+    const uint32_t o_dst =
+        mapa_shared(smem_u32(&s.k[0][0][0]) + 4u * ((rank * 32 + (r & 31)) * kStashLd), owner);
+    const uint32_t ml_dst = mapa_shared(smem_u32(&s.v[0][0][0]) + 8u * (rank * 32 + (r & 31)), owner);
+    const uint32_t t_o = tmem + (static_cast<uint32_t>(32 * warp) << 16) + kOColP;
+    if (__all_sync(0xffffffffu, have_share)) {
+#pragma unroll
+      for (int c = 0; c < kDP / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld_32x32b_x32(t_o + 32 * c, o);
+        tmem_ld_wait();
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          st_cluster_f4(o_dst + 4u * (32 * c + 4 * v),
+                        make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                    __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3])));
+      }
+      st_cluster_f2(ml_dst, make_float2(share_m2, share_l));
+    } else {
+      // no keys in this share (or a wait gave up): weight 0 in the combine
+#pragma unroll
+      for (int v = 0; v < kDP / 4; ++v) st_cluster_f4(o_dst + 16u * v, make_float4(0.0f, 0.0f, 0.0f, 0.0f));
+      st_cluster_f2(ml_dst, make_float2(-INFINITY, 0.0f));
+    }
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarpP) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  if (n_chunks > 1) {
-    // the last CTA of this query tile to finish combines the chunks in chunk
-    // order (M2 = max m2, w = 2^(m2 - M2), O = sum w acc / sum w l) and returns
-    // the ticket to zero for the next launch.  The block barrier above orders
-    // every thread's partial stores before thread 0's release fence and ticket.
-    const int64_t tile_id = (int64_t)(p.tile_start[b] + qt) * p.kv_heads + kvh;
-    if (threadIdx.x == 0) {
-      __threadfence();
-      s.last = atomicAdd(p.tickets + tile_id, 1u) == static_cast<uint32_t>(n_chunks - 1);
-      __threadfence();
-    }
-    __syncthreads();
-    if (s.last) {
-      if (warp < 4) {
-        const int r = 32 * warp + lane;
-        const int tok = tok0 + r / G;
-        const float2* ml = reinterpret_cast<const float2*>(p.part_ml);
-        const int64_t base = ((int64_t)item0 * p.kv_heads + kvh) * kQTile + r;  // chunk 0 of this row
-        const int64_t step = (int64_t)p.kv_heads * kQTile;                      // next chunk
-        float M2 = -INFINITY;
-        for (int c = 0; c < n_chunks; ++c) M2 = fmaxf(M2, __ldcg(&ml[base + c * step].x));
-        if (tok < q_len) {
-          float a[kDP];
+  // ---- the cluster's combine: after the barrier this CTA holds, for its rows
+  // [32 rank, 32 rank + 32), the four shares in rank order:
+  // M2 = max m2, w = 2^(m2 - M2), O = sum w acc / sum w l
+  cluster_sync();
+  if (warp < 4) {
+    const int row = 32 * rank + lane;  // a warp's lanes take the 32 rows, the warp a quarter of the head dim
+    const int d0 = 32 * warp;
+    const int tok = tok0 + row / G;
+    const float* slots = reinterpret_cast<const float*>(&s.k[0][0][0]);
+    const float2* slot_ml = reinterpret_cast<const float2*>(&s.v[0][0][0]);
+    float2 e[kClusterP];
 #pragma unroll
-          for (int i = 0; i < kDP; ++i) a[i] = 0.0f;
-          float Ls = 0.0f;
-          for (int c = 0; c < n_chunks; ++c) {
-            const float2 e = __ldcg(&ml[base + c * step]);
-            const float w = ex2_approx(__fsub_rn(e.x, M2));
-            Ls = __fmaf_rn(w, e.y, Ls);
-            const float4* src = reinterpret_cast<const float4*>(p.part_acc + (base + c * step) * kDP);
-            float4 x[kDP / 4];
+    for (int c = 0; c < kClusterP; ++c) e[c] = slot_ml[c * 32 + lane];
+    float M2 = -INFINITY;
 #pragma unroll
-            for (int v = 0; v < kDP / 4; ++v) x[v] = __ldcg(src + v);  // the chunk's row: 32 loads in flight
+    for (int c = 0; c < kClusterP; ++c) M2 = fmaxf(M2, e[c].x);
+    float a[32];
 #pragma unroll
-            for (int v = 0; v < kDP / 4; ++v) {
-              a[4 * v] = __fmaf_rn(w, x[v].x, a[4 * v]);
-              a[4 * v + 1] = __fmaf_rn(w, x[v].y, a[4 * v + 1]);
-              a[4 * v + 2] = __fmaf_rn(w, x[v].z, a[4 * v + 2]);
-              a[4 * v + 3] = __fmaf_rn(w, x[v].w, a[4 * v + 3]);
-            }
-          }
-          const float rl = __frcp_rn(Ls);
-          uint4* d4 = reinterpret_cast<uint4*>(p.out + ((int64_t)(p.q_off[b] + tok) * p.q_heads + kvh * G + r % G) * kDP);
+    for (int i = 0; i < 32; ++i) a[i] = 0.0f;
+    float Ls = 0.0f;
 #pragma unroll
-          for (int v = 0; v < kDP / 8; ++v) {
-            uint32_t w4[4];
+    for (int c = 0; c < kClusterP; ++c) {
+      const float w = ex2_approx(__fsub_rn(e[c].x, M2));  // 0 for a share with no keys
+      Ls = __fmaf_rn(w, e[c].y, Ls);
+      const float4* src = reinterpret_cast<const float4*>(slots + (c * 32 + lane) * kStashLd + d0);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              w4[k] = bf16x2(__fmul_rn(a[8 * v + 2 * k], rl), __fmul_rn(a[8 * v + 2 * k + 1], rl));
-            d4[v] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-          }
-        }
+      for (int v = 0; v < 8; ++v) {
+        const float4 x = src[v];
+        a[4 * v] = __fmaf_rn(w, x.x, a[4 * v]);
+        a[4 * v + 1] = __fmaf_rn(w, x.y, a[4 * v + 1]);
+        a[4 * v + 2] = __fmaf_rn(w, x.z, a[4 * v + 2]);
+        a[4 * v + 3] = __fmaf_rn(w, x.w, a[4 * v + 3]);
       }
-      if (threadIdx.x == 0) p.tickets[tile_id] = 0u;
+    }
+    if (tok < q_len) {
+      // one reciprocal per row: x * RN(1/l) is within 1.5 fp32 ulp of x / l, far
+      // below the bf16 rounding that follows
+      const float rl = __frcp_rn(Ls);
+      uint4* d4 = reinterpret_cast<uint4*>(p.out + ((int64_t)(p.q_off[b] + tok) * p.q_heads + kvh * G + row % G) * kDP +
+                                           d0);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        uint32_t w4[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          w4[k] = bf16x2(__fmul_rn(a[8 * v + 2 * k], rl), __fmul_rn(a[8 * v + 2 * k + 1], rl));
+        d4[v] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
     }
   }
 }
@@ -511,58 +496,8 @@ bool make_map_rows(CUtensorMap* m, const void* base, int64_t rows, int heads, in
 
 }  // namespace
 
-namespace {
-constexpr int kPrefillSplitKeys = 2048;  // keys per chunk: longer key ranges are split over CTAs
-
-struct PrefillLaunch {  // one launch: sequences [s0, s0 + n)
-  int32_t s0, n, tiles, items;
-};
-
-inline size_t al1k(size_t x) { return (x + 1023) / 1024 * 1024; }
-
-// Tiles and work items of the launches covering all sequences.
-std::vector<PrefillLaunch> plan_prefill(const PrefillSeq* seqs, int32_t n_seqs, int32_t tpt, int32_t causal) {
-  std::vector<PrefillLaunch> out;
-  for (int32_t s0 = 0; s0 < n_seqs; s0 += kPrefillMaxSeqs) {
-    PrefillLaunch l{s0, n_seqs - s0 < kPrefillMaxSeqs ? n_seqs - s0 : kPrefillMaxSeqs, 0, 0};
-    for (int32_t i = 0; i < l.n; ++i) {
-      const PrefillSeq& q = seqs[s0 + i];
-      const int64_t nt = (q.q_len + tpt - 1) / tpt;
-      for (int64_t t = 0; t < nt; ++t) {
-        const int64_t te = (t + 1) * tpt < q.q_len ? (t + 1) * tpt : q.q_len;
-        const int64_t keys = causal ? q.kv_len - q.q_len + te : q.kv_len;
-        l.items += static_cast<int32_t>((keys + kPrefillSplitKeys - 1) / kPrefillSplitKeys);
-      }
-      l.tiles += static_cast<int32_t>(nt);
-    }
-    out.push_back(l);
-  }
-  return out;
-}
-
-// Scratch after the 256-byte error word: tickets, then the chunk partials.
-struct PrefillScratch {
-  size_t tickets, ml, acc, total;
-};
-PrefillScratch prefill_scratch(int32_t tiles, int32_t items, int32_t kv_heads) {
-  PrefillScratch w;
-  w.tickets = 256;
-  w.ml = al1k(w.tickets + (size_t)tiles * kv_heads * sizeof(uint32_t));
-  w.acc = al1k(w.ml + (size_t)items * kv_heads * kQTile * 2 * sizeof(float));
-  w.total = al1k(w.acc + (size_t)items * kv_heads * kQTile * kDP * sizeof(float));
-  return w;
-}
-}  // namespace
-
-size_t gqa_prefill_ws_bytes(const PrefillSeq* seqs, int32_t n_seqs, int32_t q_heads, int32_t kv_heads,
-                            int32_t causal) {
-  const int32_t tpt = kQTile / (q_heads / kv_heads);
-  size_t need = 256;
-  for (const PrefillLaunch& l : plan_prefill(seqs, n_seqs, tpt, causal)) {
-    const size_t t = prefill_scratch(l.tiles, l.items, kv_heads).total;
-    need = t > need ? t : need;
-  }
-  return need;
+size_t gqa_prefill_ws_bytes(const PrefillSeq*, int32_t, int32_t, int32_t, int32_t) {
+  return 256;  // the error word: the split of a tile's keys is combined on chip
 }
 
 cudaError_t launch_gqa_prefill(const void* q, const void* k, const void* v, int64_t total_q, int64_t total_kv,
@@ -578,43 +513,31 @@ cudaError_t launch_gqa_prefill(const void* q, const void* k, const void* v, int6
   cudaError_t e = cudaFuncSetAttribute(gqa_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  for (const PrefillLaunch& l : plan_prefill(seqs, n_seqs, tpt, causal)) {
-    if (l.items == 0) continue;
-    const PrefillScratch w = prefill_scratch(l.tiles, l.items, kv_heads);
+  for (int32_t s0 = 0; s0 < n_seqs; s0 += kPrefillMaxSeqs) {
     PrefillParams p;
-    p.n_seqs = l.n;
+    p.n_seqs = n_seqs - s0 < kPrefillMaxSeqs ? n_seqs - s0 : kPrefillMaxSeqs;
     p.q_heads = q_heads;
     p.kv_heads = kv_heads;
     p.group = G;
     p.tokens_per_tile = tpt;
     p.causal = causal;
-    p.split_keys = kPrefillSplitKeys;
     p.c2 = 0.12751743074419465f;  // log2(e) / sqrt(128)
     p.out = reinterpret_cast<__nv_bfloat16*>(out);
     p.err = reinterpret_cast<uint32_t*>(ws);
-    p.tickets = reinterpret_cast<uint32_t*>(ws + w.tickets);
-    p.part_ml = reinterpret_cast<float*>(ws + w.ml);
-    p.part_acc = reinterpret_cast<float*>(ws + w.acc);
-    int tiles = 0, items = 0;
-    for (int i = 0; i < l.n; ++i) {
-      const PrefillSeq& sq = seqs[l.s0 + i];
+    int tiles = 0;
+    for (int i = 0; i < p.n_seqs; ++i) {
+      const PrefillSeq& sq = seqs[s0 + i];
       p.q_off[i] = static_cast<int32_t>(sq.q_off);
       p.q_len[i] = static_cast<int32_t>(sq.q_len);
       p.kv_off[i] = static_cast<int32_t>(sq.kv_off);
       p.kv_len[i] = static_cast<int32_t>(sq.kv_len);
       p.tile_start[i] = tiles;
-      p.item_start[i] = items;
-      const int nt = static_cast<int>((sq.q_len + tpt - 1) / tpt);
-      for (int t = 0; t < nt; ++t) {
-        const int64_t te = (int64_t)(t + 1) * tpt < sq.q_len ? (int64_t)(t + 1) * tpt : sq.q_len;
-        const int64_t keys = causal ? sq.kv_len - sq.q_len + te : sq.kv_len;
-        items += static_cast<int>((keys + kPrefillSplitKeys - 1) / kPrefillSplitKeys);
-      }
-      tiles += nt;
+      tiles += static_cast<int>((sq.q_len + tpt - 1) / tpt);
     }
-    p.tile_start[l.n] = tiles;
-    p.item_start[l.n] = items;
-    dim3 grid(static_cast<unsigned>(items), static_cast<unsigned>(kv_heads));
+    p.tile_start[p.n_seqs] = tiles;
+    if (tiles == 0) continue;
+    // one cluster of kClusterP CTAs per (query tile, key/value head)
+    dim3 grid(static_cast<unsigned>(tiles * kClusterP), static_cast<unsigned>(kv_heads));
     gqa_prefill_kernel<<<grid, kThreadsP, smem, st>>>(tq, tk, tv, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -309,11 +309,10 @@ sdm_status sdm_cached_attention_offload(const void* q, int32_t batch, int64_t n_
  *   qo_indptr, kv_indptr  HOST arrays of batch + 1 int64 offsets, starting at 0
  *   out  [total_q][q_heads][128] bf16
  *   q_heads / kv_heads in {1, 2, 4, 8, 16}; head_dim 128 (else SDM_ERR_UNSUPPORTED)
- *   ws   >= sdm_gqa_prefill_workspace_size(...) bytes, all zero before its first
- *        use: the error word, one ticket per (query tile, key/value head) --
- *        the kernel returns them to zero -- and the partial results of the
- *        256-key chunks a query tile's keys are split into (the last CTA of a
- *        tile to finish combines them in chunk order).
+ *   ws   >= sdm_gqa_prefill_workspace_size(...) bytes (the error word; its first
+ *        256 bytes zero before first use).  A query tile's keys are split over
+ *        a cluster of 4 CTAs that combine their shares in shared memory, in
+ *        rank order, so the result does not depend on timing.
  * This entry point has no counterpart on the pages that define the ICL layer.
  */
 size_t sdm_gqa_prefill_workspace_size(const int64_t* qo_indptr, const int64_t* kv_indptr, int32_t batch,

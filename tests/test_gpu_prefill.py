@@ -77,7 +77,7 @@ def test_prefill_contract_shape(cuda_lib, orc, causal):
 
 @pytest.mark.parametrize("q_lens,kv_lens", [((1, 17, 100), (1, 300, 1000)), ((5, 0, 33), (5, 7, 33)),
                                             ((129,), (129,)), ((40, 31), (2000, 31)),
-                                            ((50, 3), (5000, 4200))])   # key ranges split over CTAs
+                                            ((50, 3), (5000, 4200))])   # long key ranges
 def test_prefill_ragged_lengths(cuda_lib, orc, q_lens, kv_lens):
     inp = make_prefill_inputs(W, q_lens=q_lens, kv_lens=kv_lens)
     check(cuda_lib, orc, inp, True, f"ragged q{q_lens} kv{kv_lens}")
@@ -111,7 +111,7 @@ def test_prefill_is_deterministic_and_leaves_no_error(cuda_lib):
 
 
 def test_prefill_workspace_reuse_across_batches(cuda_lib, orc):
-    """One workspace for several different batches in a row: the tickets go back to zero."""
+    """One workspace for several different batches in a row."""
     shapes = [((50, 3), (5000, 4200)), ((1, 17, 100), (1, 300, 1000)), ((50, 3), (5000, 4200))]
     need = max(cuda_lib.gqa_prefill_workspace_size(np.concatenate([[0], np.cumsum(ql)]),
                                                    np.concatenate([[0], np.cumsum(kl)]), 16, 4) for ql, kl in shapes)
