@@ -564,7 +564,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, help="workload name (profiling runs use smaller ones)")
-    ap.add_argument("--cpu-rows", type=int, default=64, help="rows of the oracle's timed sample")
+    ap.add_argument("--cpu-rows", type=int, default=640,
+                    help="rows of the oracle's timed sample (about 10 s of host-core work at 512K)")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--per-kernel", action="store_true",
