@@ -65,6 +65,11 @@ __device__ __forceinline__ uint32_t o_col(int t) { return 128u * kTiles + 80u * 
 template <int kTiles>
 __device__ __forceinline__ uint32_t p_col(int t) { return 208u * kTiles + 32u * t; }
 
+// log2 of the largest probability a skipped tile may hold: e4m3 rounds
+// everything at or below 2^-10 to zero, so 2^-11 leaves room for the error of
+// the hardware 2^x and of the polynomial.
+constexpr float kDeadExponent = -11.0f;
+
 constexpr long long kWaitLimit = 1LL << 31;   // ~1 s of SM clock: no legitimate wait comes close
 constexpr long long kDrainLimit = 1LL << 24;  // teardown waits for copies in flight
 
@@ -344,6 +349,7 @@ __global__ void __launch_bounds__(Cfg<kTiles>::kThreads, Cfg<kTiles>::kMinBlocks
     const bool warp_rows = kTiles == 1 ? (row0 + 32 * wq < p.T) : true;
     float m_run = -INFINITY;  // running max of raw z
     float m2 = -INFINITY;     // fp32(m_run * c2)
+    bool p_zero = false;      // this warp's P_t columns hold e4m3 zeros
     bool ok = true;
     for (int it = 0; it < n_tiles; ++it) {
       ok = mbar_wait(&s.s_full[t], it & 1, abort_flag, kWaitLimit);
@@ -390,7 +396,7 @@ __global__ void __launch_bounds__(Cfg<kTiles>::kThreads, Cfg<kTiles>::kMinBlocks
         mask_keys(ra, rb, 0, nvalid);
         mask_keys(rc, rd, 64, nvalid);
       }
-      float mx0 = m_run, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         if (i % 2 == 0) {
@@ -401,11 +407,45 @@ __global__ void __launch_bounds__(Cfg<kTiles>::kThreads, Cfg<kTiles>::kMinBlocks
           mx3 = max3(mx3, __uint_as_float(rc[i]), __uint_as_float(rd[i]));
         }
       }
-      const float mt = max3(mx0, mx1, fmaxf(mx2, mx3));
+      const float mtile = max3(mx0, mx1, fmaxf(mx2, mx3));  // this tile's largest logit
+      const float mt = fmaxf(m_run, mtile);
       const bool up = mt > m_run;
       const float m2_new = up ? __fmul_rn(mt, c2) : m2;
       // P = 2^(fma(z, c2, -m2)) in (0, 1] -> e4m3, four codes per 32-bit TMEM column
       const float nm2 = -m2_new;
+      // At or below 2^-10 every probability rounds to the e4m3 zero, through
+      // ex2.approx and through the polynomial alike. fma is monotone in z
+      // (c2 > 0), so if the tile's largest logit lands below 2^-11 in every row
+      // of the warp, all of this warp's P_t is zero: skip the 2^x work and store
+      // zeros, or nothing if the columns already hold zeros. The P V product
+      // still runs and adds exact zeros, so the result is the same to the bit.
+      // (Such a tile cannot raise the running max, so m_run and m2 stay.)
+      // The arrival on p_full must not come before the previous tile's phase
+      // has completed, or a fast warp would count twice toward it: a store
+      // waits for the previous P V as the dense path does; without a store
+      // the warp waits for the previous P_t to be complete.
+      if (__all_sync(0xffffffffu, __fmaf_rn(mtile, c2, nm2) < kDeadExponent)) {
+        if (it > 0) {
+          ok = p_zero ? mbar_wait(&s.p_full[t], (it - 1) & 1, abort_flag, kWaitLimit)
+                      : mbar_wait(&s.o_ready[t], (it - 1) & 1, abort_flag, kWaitLimit);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) {
+            if (lane == 0) raise_abort(s, p.err, p_zero ? kErrTimeoutP : kErrTimeoutO);
+            break;
+          }
+          tc_fence_after();
+        }
+        if (!p_zero) {
+          tmem_st_32x32b_x32_zero(t_p);
+          tmem_st_wait();
+          p_zero = true;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.p_full[t]);
+        continue;
+      }
+      p_zero = false;
       {
         uint32_t pw[32];
         p_words32<0>(ra, rb, rc, rd, pw, c2, nm2);

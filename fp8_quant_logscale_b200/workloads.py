@@ -63,6 +63,11 @@ WORKLOADS = {
     "icl_n512k_m1k_h8": Workload(
         "icl_n512k_m1k_h8", 524288, 1024, 8, seed=4,
         description="N=524288, M=1024, H=8, d=64, fp16 N(0,1); LogScale; FP8 self + cross attention"),
+    "icl_n128k_m1k_h8_flat": Workload(
+        "icl_n128k_m1k_h8_flat", 131072, 1024, 8, head_factor=(0.01, 0.02), seed=8,
+        description="N=131072, M=1024, H=8, d=64, fp16 N(0,1) scaled per (tensor, head) by U(0.01,0.02): "
+                    "logits within a fraction of a unit, so every key keeps a non-zero e4m3 probability "
+                    "(the dense-softmax case of the FP8 attention); LogScale"),
     "final_n8k_m1k_h8_gated": Workload(
         "final_n8k_m1k_h8_gated", 8192, 1024, 8, head_factor=(0.5, 4.0), gated=True, seed=6,
         description="N=8192, M=1024, H=8, d=64, fp16 N(0,1) scaled per (tensor, head) by U(0.5,4); "
