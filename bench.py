@@ -42,8 +42,8 @@ BF16_NOMINAL_TFLOPS = 2250.0
 # Valid only for the kernel source it was taken on: any change to these files
 # makes the bench report null until a new capture is recorded here.
 ATTN_TRAFFIC_SOURCES = ("attention.cu", "ptx.cuh", "exp2_poly.cuh", "kernels.cuh", "softmax.cuh")
-ATTN_TRAFFIC = {"source_sha256": "cb4639859d9ea0e3e81f0ad51963284513f69bbc6cede5ed0eb8c7a8c96bd1f1",
-                "bytes": 6.25e9 + 592.16e6}
+ATTN_TRAFFIC = {"source_sha256": "5acf03581f9db5d1bcd7257eb1d477e6ede4ffb448c69588f4521564c0f1f861",
+                "bytes": 5.878e9 + 629.87e6}
 
 
 def attention_source_sha256() -> str:
@@ -319,7 +319,10 @@ def run_ours(args):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
                      "frac": achieved / fp8_peak, "traffic": traffic, "peak_source": peak_src,
                      "kernel": "icl_attention_kernel (FP8 attention of all rows)"},
-        "softmax_bound": {"kind": "MUFU ex2, 16/clk/SM, one per logit", "peak": mufu_tflops, "unit": "TFLOP/s",
+        # warp tiles whose probabilities all round to the e4m3 zero skip their 2^x,
+        # so on peaked attention this bound of the dense softmax can be exceeded
+        "softmax_bound": {"kind": "MUFU ex2, 16/clk/SM, one per logit of the dense softmax (exact-zero tiles "
+                                  "skip theirs)", "peak": mufu_tflops, "unit": "TFLOP/s",
                           "frac": achieved / mufu_tflops, "sm_mhz": mhz, "sms": sms},
         "gpu_launches": args.steps * 9,
         "clocks": clocks,
