@@ -465,19 +465,27 @@ __global__ void __launch_bounds__(Cfg<kTiles>::kThreads, Cfg<kTiles>::kMinBlocks
       if (it > 0 && __any_sync(0xffffffffu, up)) {
         // O and its row sum were accumulated against the old max: rescale (after
         // the P stores, so the logits' registers are free again).
+        // One TMEM round trip: the 64 columns of O and the row sum are loaded
+        // together (the logits' registers are free again), scaled with packed
+        // multiplies and stored back.
         const float alpha = up ? ex2_approx(__fsub_rn(m2, m2_new)) : 1.0f;
-        uint32_t o[32];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          tmem_ld_32x32b_x32(t_o + 32 * c, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__fmul_rn(__uint_as_float(o[i]), alpha));
-          tmem_st_32x32b_x32(t_o + 32 * c, o);
-        }
-        uint32_t l;
+        uint32_t o0[32], o1[32], l;
+        tmem_ld_32x32b_x32(t_o, o0);
+        tmem_ld_32x32b_x32(t_o + 32, o1);
         tmem_ld_32x32b_x1(t_o + kHeadDim, l);
         tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float a0, a1, b0, b1;
+          mul2(a0, a1, __uint_as_float(o0[i]), __uint_as_float(o0[i + 1]), alpha, alpha);
+          mul2(b0, b1, __uint_as_float(o1[i]), __uint_as_float(o1[i + 1]), alpha, alpha);
+          o0[i] = __float_as_uint(a0);
+          o0[i + 1] = __float_as_uint(a1);
+          o1[i] = __float_as_uint(b0);
+          o1[i + 1] = __float_as_uint(b1);
+        }
+        tmem_st_32x32b_x32(t_o, o0);
+        tmem_st_32x32b_x32(t_o + 32, o1);
         tmem_st_32x32b_x1(t_o + kHeadDim, __float_as_uint(__fmul_rn(__uint_as_float(l), alpha)));
       }
       m_run = mt;
