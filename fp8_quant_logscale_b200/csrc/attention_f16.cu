@@ -334,15 +334,23 @@ __global__ void __launch_bounds__(kThreadsH, 1)
         tmem_st_32x32b_x32(t_p + 32, pa);
       }
       if (it > 0 && __any_sync(0xffffffffu, up)) {
-        uint32_t o[32];
+        // both halves of O in one TMEM round trip, packed multiplies
+        uint32_t o0[32], o1[32];
+        tmem_ld_32x32b_x32(t_o, o0);
+        tmem_ld_32x32b_x32(t_o + 32, o1);
+        tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          tmem_ld_32x32b_x32(t_o + 32 * c, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__fmul_rn(__uint_as_float(o[i]), alpha));
-          tmem_st_32x32b_x32(t_o + 32 * c, o);
+        for (int i = 0; i < 32; i += 2) {
+          float a0, a1, b0, b1;
+          mul2(a0, a1, __uint_as_float(o0[i]), __uint_as_float(o0[i + 1]), alpha, alpha);
+          mul2(b0, b1, __uint_as_float(o1[i]), __uint_as_float(o1[i + 1]), alpha, alpha);
+          o0[i] = __float_as_uint(a0);
+          o0[i + 1] = __float_as_uint(a1);
+          o1[i] = __float_as_uint(b0);
+          o1[i + 1] = __float_as_uint(b1);
         }
+        tmem_st_32x32b_x32(t_o, o0);
+        tmem_st_32x32b_x32(t_o + 32, o1);
       }
       m_run = mt;
       m2 = m2_new;
