@@ -578,6 +578,9 @@ __global__ void __launch_bounds__(Cfg<kTiles>::kThreads, Cfg<kTiles>::kMinBlocks
 // ------------------------------------------------------------ split-KV reduce
 // One warp per (b, h, row): M2 = max_s m2_s; w_s = 2^(m2_s - M2);
 // O = (sum_s w_s acc_s) * s_v / (sum_s w_s l_s), splits in ascending order.
+// Lane j fetches the (m2, l) pair of split s0 + j; the weights reach every lane
+// by shuffles, and each lane loads eight splits of its two accumulator columns
+// ahead of the multiply-adds, which still run one split after another.
 __global__ void __launch_bounds__(256) splitkv_reduce_kernel(const float* __restrict__ part_acc,
                                                              const float* __restrict__ part_ml, int64_t n_splits,
                                                              int32_t BH, int32_t H, int64_t T,
@@ -587,17 +590,36 @@ __global__ void __launch_bounds__(256) splitkv_reduce_kernel(const float* __rest
   if (gw >= (int64_t)BH * T) return;
   const int64_t bh = gw / T, row = gw % T;
   const float2* ml = reinterpret_cast<const float2*>(part_ml);
+  const float2* acc2 = reinterpret_cast<const float2*>(part_acc);
   float M2 = -INFINITY;
-  for (int64_t sidx = 0; sidx < n_splits; ++sidx) M2 = fmaxf(M2, ml[(sidx * BH + bh) * T + row].x);
+  for (int64_t s0 = lane; s0 < n_splits; s0 += 32) M2 = fmaxf(M2, ml[(s0 * BH + bh) * T + row].x);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M2 = fmaxf(M2, __shfl_xor_sync(0xffffffffu, M2, o));
   float L = 0.0f, a0 = 0.0f, a1 = 0.0f;
-  for (int64_t sidx = 0; sidx < n_splits; ++sidx) {
-    const int64_t prow = (sidx * BH + bh) * T + row;
-    const float2 e = ml[prow];
-    const float w = ex2_approx(__fsub_rn(e.x, M2));
-    const float2 acc = reinterpret_cast<const float2*>(part_acc + prow * kHeadDim)[lane];
-    L = __fmaf_rn(w, e.y, L);
-    a0 = __fmaf_rn(w, acc.x, a0);
-    a1 = __fmaf_rn(w, acc.y, a1);
+  for (int64_t s0 = 0; s0 < n_splits; s0 += 32) {
+    const int cnt = n_splits - s0 < 32 ? static_cast<int>(n_splits - s0) : 32;
+    float w = 0.0f, lv = 0.0f;
+    if (lane < cnt) {
+      const float2 e = ml[((s0 + lane) * BH + bh) * T + row];
+      w = ex2_approx(__fsub_rn(e.x, M2));
+      lv = e.y;
+    }
+    for (int j = 0; j < cnt; j += 8) {
+      float2 acc[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (j + u < cnt) acc[u] = acc2[(((s0 + j + u) * BH + bh) * T + row) * (kHeadDim / 2) + lane];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (j + u < cnt) {
+          const float ws = __shfl_sync(0xffffffffu, w, j + u);
+          const float ls = __shfl_sync(0xffffffffu, lv, j + u);
+          L = __fmaf_rn(ws, ls, L);
+          a0 = __fmaf_rn(ws, acc[u].x, a0);
+          a1 = __fmaf_rn(ws, acc[u].y, a1);
+        }
+      }
+    }
   }
   const float s_v = __ldg(scales + 2 * BH + bh);
   const int64_t b = bh / H, h = bh % H;
