@@ -1,0 +1,105 @@
+"""GPU parity on inputs built so that whole 128-key tiles hold only e4m3-zero
+probabilities.
+
+Every row shares one direction u with the keys of two "hot" tiles, so the row
+maxima sit in those tiles and the other keys lie hundreds of log2 units below
+them: their probabilities round to the e4m3 zero.  The FP8 attention kernel
+skips the 2^x work of such tiles; these inputs make it take each branch of that
+skip -- the first skipped tile (zeros stored), the skipped tiles after it
+(nothing stored), a live tile after a run of skipped ones, a ragged last tile --
+on the one-call path and on split-KV chunks (which restart the running max).
+Outputs must match the oracle within the specification's gates, like any other
+input.
+"""
+import numpy as np
+import pytest
+
+from parity import DELTA, dev, gate, host
+
+pytestmark = pytest.mark.gpu
+LOG2E = 1.4426950408889634
+HOT = (3, 9)
+
+
+def _f16(x):
+    return np.asarray(x, np.float32).astype(np.float16)
+
+
+def _hot_tile_inputs(N=2000, M=160, H=2, seed=21):
+    rng = np.random.default_rng(seed)
+    T = N + M
+    u = rng.choice([-1.0, 1.0], size=(H, 64))
+    q = 2.0 * u[None, None] + 0.3 * rng.standard_normal((1, T, H, 64))
+    k = 0.3 * rng.standard_normal((1, N, H, 64))
+    for j in HOT:
+        k[:, 128 * j:128 * (j + 1)] += 2.0 * u[None, None]
+    v = rng.standard_normal((1, N, H, 64))
+    return dict(q=_f16(q), k=_f16(k), v=_f16(v), c_h=np.ones(H, np.float32), B=1, N=N, M=M, H=H)
+
+
+def _dead_warp_tiles(orc, inp, split):
+    """[H, row warps, key tiles] bool: every row of a 32-row warp has the tile's
+    largest logit more than 11.5 log2 units below its running max (a margin over
+    the kernel's 11), computed in float64 from the oracle's FP8 codes; key tiles
+    restart their running max at every split-KV chunk boundary."""
+    N = inp["N"]
+    qs = orc.qscale(inp["q"], N, inp["c_h"])
+    s_q, s_k = orc.context_scales(qs, N), orc.context_scales(inp["k"], N)
+    q = orc.e4m3_decode(orc.quantize(qs, s_q))[0].astype(np.float64)      # [H, T, d]
+    k = orc.e4m3_decode(orc.quantize(inp["k"], s_k))[0].astype(np.float64)
+    T, n_tiles = q.shape[1], (N + 127) // 128
+    out = []
+    for h in range(inp["H"]):
+        c2 = float(s_q[0, h]) * float(s_k[0, h]) * LOG2E / 8.0
+        z = q[h] @ k[h].T                                                  # [T, N]
+        zt = np.full((T, n_tiles * 128), -np.inf)
+        zt[:, :N] = z
+        tmax = zt.reshape(T, n_tiles, 128).max(axis=2)
+        run = np.empty_like(tmax)
+        for j in range(n_tiles):
+            fresh = split and (j * 128) % split == 0
+            run[:, j] = tmax[:, j] if (j == 0 or fresh) else np.maximum(run[:, j - 1], tmax[:, j])
+        dead = (tmax - run) * c2 < -11.5
+        w = T // 32
+        out.append(dead[:w * 32].reshape(w, 32, n_tiles).all(axis=1))
+    return np.array(out)
+
+
+def test_zero_tiles_one_call(cuda_lib, orc):
+    inp = _hot_tile_inputs()
+    N, M, H = inp["N"], inp["M"], inp["H"]
+    dead = _dead_warp_tiles(orc, inp, split=0)
+    # the construction reaches every branch of the skip, in every row warp
+    assert dead[:, :, HOT[0] + 1:HOT[1]].all(), "tiles between the hot ones are skipped"
+    assert not dead[:, :, HOT[1]].any(), "the second hot tile is live again"
+    assert dead[:, :, -1].all(), "the ragged last tile is skipped"
+    cache = cuda_lib.FP8Cache(1, N, H, "cuda")
+    ws = cuda_lib.new_workspace(cuda_lib.workspace_size(1, 1, N, M, H, keep_cache=True), "cuda")
+    out = cuda_lib.icl_attention(dev(inp["q"]), dev(inp["k"]), dev(inp["v"]), N, dev(inp["c_h"]), cache=cache,
+                                 ws=ws)
+    st, flags = cuda_lib.sync_status(ws)
+    assert st == 0 and flags == 0, (st, flags)
+    ref = orc.layer(inp["q"], inp["k"], inp["v"], N, inp["c_h"], delta=DELTA)
+    stats = gate(host(out), ref["out"], ref["allow"], "zero tiles, one call")
+    print(f"\nzero tiles one call: {stats}")
+
+
+def test_zero_tiles_split_kv(cuda_lib, orc):
+    inp = _hot_tile_inputs()
+    N, M, H = inp["N"], inp["M"], inp["H"]
+    split = orc.split_keys(N)
+    dead = _dead_warp_tiles(orc, inp, split=split)
+    # the second chunk starts fresh on a cold tile (live), then its hot tile raises the max
+    first = split // 128
+    assert not dead[:, :, first].any() and dead[:, :, HOT[1] + 1:].all()
+    cache = cuda_lib.FP8Cache(1, N, H, "cuda")
+    cuda_lib.icl_attention(dev(inp["q"]), dev(inp["k"]), dev(inp["v"]), N, dev(inp["c_h"]), cache=cache)
+    queries = inp["q"][:, N:]
+    pred = host(cuda_lib.cached_attention(dev(queries), cache, dev(inp["c_h"])))
+    qs = orc.qscale(inp["q"], N, inp["c_h"])
+    s_q, s_k, s_v = (orc.context_scales(x, N) for x in (qs, inp["k"], inp["v"]))
+    k8, v8 = orc.quantize(inp["k"], s_k), orc.quantize(inp["v"], s_v)
+    qq = orc.quantize(orc.qscale(queries, N, inp["c_h"]), s_q)
+    _, o, allow = orc.attention(qq, k8, v8, s_q, s_k, s_v, split=split, delta=DELTA)
+    stats = gate(pred, o, allow, "zero tiles, split-KV")
+    print(f"\nzero tiles split-KV: {stats}")
