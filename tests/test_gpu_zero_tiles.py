@@ -84,7 +84,9 @@ def test_zero_tiles_one_call(cuda_lib, orc):
     print(f"\nzero tiles one call: {stats}")
 
 
-def test_zero_tiles_split_kv(cuda_lib, orc):
+@pytest.mark.parametrize("n_pred", [160, 64])
+def test_zero_tiles_split_kv(cuda_lib, orc, n_pred):
+    """160 queries run on the two-tile kernel, 64 on the one-tile kernel of small batches."""
     inp = _hot_tile_inputs()
     N, M, H = inp["N"], inp["M"], inp["H"]
     split = orc.split_keys(N)
@@ -94,12 +96,12 @@ def test_zero_tiles_split_kv(cuda_lib, orc):
     assert not dead[:, :, first].any() and dead[:, :, HOT[1] + 1:].all()
     cache = cuda_lib.FP8Cache(1, N, H, "cuda")
     cuda_lib.icl_attention(dev(inp["q"]), dev(inp["k"]), dev(inp["v"]), N, dev(inp["c_h"]), cache=cache)
-    queries = inp["q"][:, N:]
+    queries = np.ascontiguousarray(inp["q"][:, N:N + n_pred])
     pred = host(cuda_lib.cached_attention(dev(queries), cache, dev(inp["c_h"])))
     qs = orc.qscale(inp["q"], N, inp["c_h"])
     s_q, s_k, s_v = (orc.context_scales(x, N) for x in (qs, inp["k"], inp["v"]))
     k8, v8 = orc.quantize(inp["k"], s_k), orc.quantize(inp["v"], s_v)
     qq = orc.quantize(orc.qscale(queries, N, inp["c_h"]), s_q)
     _, o, allow = orc.attention(qq, k8, v8, s_q, s_k, s_v, split=split, delta=DELTA)
-    stats = gate(pred, o, allow, "zero tiles, split-KV")
-    print(f"\nzero tiles split-KV: {stats}")
+    stats = gate(pred, o, allow, f"zero tiles, split-KV, {n_pred} queries")
+    print(f"\nzero tiles split-KV, {n_pred} queries: {stats}")
