@@ -38,7 +38,7 @@ BF16_NOMINAL_TFLOPS = 2250.0
 
 
 # DRAM bytes (read + write) of one fit launch of the attention kernel on the
-# 512K workload, from a one-pass ncu capture (profiles/icl_attention_kernel_n512k_dram.md).
+# 512K workload, from a one-pass ncu capture (dram__bytes_read.sum + dram__bytes_write.sum).
 # Valid only for the kernel source it was taken on: any change to these files
 # makes the bench report null until a new capture is recorded here.
 ATTN_TRAFFIC_SOURCES = ("attention.cu", "ptx.cuh", "exp2_poly.cuh", "kernels.cuh", "softmax.cuh")

@@ -8,7 +8,7 @@ into TabICLv2", timing table: 16,384 to 524,288 context rows, 1,024 query
 rows); none of that is available, so these seeded tensors of the same shapes
 stand in for the attention layer's Q/K/V.
 
-Generation recipe (also stated in the design doc): numpy ``Generator(PCG64)``
+Generation recipe: numpy ``Generator(PCG64)``
 streams keyed by (seed, tensor id, chunk index) over 2^22-element chunks,
 standard normal in float32, rounded to fp16 (RNE); per-(tensor, head) factors
 and the 0.1% x20 outliers, where a workload asks for them, come from their own
