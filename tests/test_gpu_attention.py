@@ -63,8 +63,11 @@ def _layer_case(cuda_lib, orc, inp, gated=False, rows=None, report=""):
     o16, o, allow = orc.attention(q8, k8, v8, s_q, s_k, s_v, rows=rows, delta=DELTA)
     got = host(out) if rows is None else host(out)[:, rows]
     stats = gate(got, o, allow, report)
-    exact = orc.attention_exact(qs, inp["k"], inp["v"], rows=rows)
-    e = got.astype(np.float64) - exact
+    # error against exact attention, reported only: on at most 256 of the checked rows
+    # (the double-precision reference is the slowest part of the large cases)
+    sub = slice(None) if rows is None or len(rows) <= 256 else slice(None, None, -(-len(rows) // 256))
+    exact = orc.attention_exact(qs, inp["k"], inp["v"], rows=None if rows is None else rows[sub])
+    e = (got if rows is None else got[:, sub]).astype(np.float64) - exact
     stats["vs_exact_rel_rms"] = float(np.sqrt((e ** 2).mean() / (exact ** 2).mean()))
     print(f"\n{report}: {stats}")
     return stats
@@ -103,9 +106,10 @@ def test_layer_128k_gated_sampled(cuda_lib, orc):
 
 
 def test_layer_512k_sampled(cuda_lib, orc):
+    """The 512K workload's own check: a seeded sample of 256 context rows and every query row."""
     w = WORKLOADS["icl_n512k_m1k_h8"]
     inp = make_inputs(w)
-    _layer_case(cuda_lib, orc, inp, rows=_sample_rows(w.n_ctx, w.n_query, 64, 128, 4), report="512K")
+    _layer_case(cuda_lib, orc, inp, rows=_sample_rows(w.n_ctx, w.n_query, 256, w.n_query, 4), report="512K")
 
 
 def test_layer_max_heads(cuda_lib, orc):

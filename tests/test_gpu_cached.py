@@ -54,14 +54,13 @@ def test_batch_split_invariance_small(cuda_lib):
 
 def test_cached_512k_full_size(cuda_lib, orc):
     """The cached-prediction workload: 1,024 queries against a 524,288-row FP8 cache,
-    bitwise equal across batch splits 1/64/1024, oracle-checked on sampled queries."""
+    bitwise equal across batch splits 1/64/1024, every query checked against the oracle."""
     w = WORKLOADS["cached_n512k_m1k_h8"]
     inp = make_inputs(w)
     cache = _fit(cuda_lib, inp)
     full = _split_equal(cuda_lib, cache, dev(inp["queries"]), dev(inp["c_h"]))
-    rows = np.sort(np.random.default_rng(5).choice(w.n_query, 96, replace=False)).astype(np.int64)
-    _, o, allow = _oracle_cached(orc, inp, inp["queries"], rows=rows)
-    print("\ncached 512K:", gate(full[:, rows], o, allow, "cached 512K"))
+    _, o, allow = _oracle_cached(orc, inp, inp["queries"])
+    print("\ncached 512K:", gate(full, o, allow, "cached 512K"))
 
 
 def test_cached_batch2_gated_queries(cuda_lib, orc):
