@@ -59,3 +59,27 @@ def test_quotients_of_every_fp16_value(cuda_lib, orc):
         a = np.float32(amax[i])
         x[b, :, h, :] = np.clip(base, -a, a).astype(np.float16)
     _check(cuda_lib, orc, x, x.copy(), x.copy(), rows)
+
+
+def test_query_rows_above_the_context_amax_saturate(cuda_lib, orc):
+    """Scales come from the context rows only, so query rows larger than every
+    context value quantise to the saturated codes +-448 (0x7E / 0xFE); the codes
+    match the oracle bit for bit and the layer's outputs for those rows stay
+    within the gates."""
+    from parity import DELTA, gate
+    N, M, H = 1000, 100, 3
+    inp = make_inputs(WORKLOADS["icl_n1k_m128_h4"], n_ctx=N, n_query=M, heads=H)
+    q = inp["q"].astype(np.float32)
+    q[:, N:] *= 10.0                                           # queries up to 10x the context amax
+    q = q.astype(np.float16)
+    qs = orc.qscale(q, N, inp["c_h"])
+    s_q = orc.context_scales(qs, N)
+    want = orc.quantize(qs, s_q)
+    sat = (want[:, :, N:] & 0x7F) == 0x7E
+    assert sat.mean() > 0.2, "the construction saturates a large share of the query codes"
+    q8, cache = cuda_lib.fp8_quantize_context(dev(qs), dev(inp["k"]), dev(inp["v"]), N)
+    torch.cuda.synchronize()
+    assert (host(q8) == want).all()
+    out = cuda_lib.icl_attention(dev(q), dev(inp["k"]), dev(inp["v"]), N, dev(inp["c_h"]))
+    ref = orc.layer(q, inp["k"], inp["v"], N, inp["c_h"], delta=DELTA)
+    gate(host(out), ref["out"], ref["allow"], "saturated query rows")
