@@ -116,3 +116,16 @@ def test_layer_max_heads(cuda_lib, orc):
     """128 heads (the largest the ABI accepts), small context."""
     inp = make_inputs(WORKLOADS["icl_n1k_m128_h4"], n_ctx=200, n_query=30, heads=128)
     _layer_case(cuda_lib, orc, inp, report="H128")
+
+
+def test_layer_gate_extremes(cuda_lib, orc):
+    """GatedLogScale at its ends: g = -20 gives the factor fp16(1 + tanh g) = 0, so q' = 0 and the
+    row attends uniformly (its output is the mean of the V codes); g = +20 doubles the row."""
+    N, M, H = 1500, 300, 4
+    inp = make_inputs(WORKLOADS["icl_n1k_m128_h4"], n_ctx=N, n_query=M, heads=H)
+    rng = np.random.default_rng(9)
+    inp["gate"] = rng.choice(np.array([-20.0, -1.0, 0.0, 1.0, 20.0], np.float16), size=(1, N + M, H))
+    qs = orc.qscale(inp["q"], N, inp["c_h"], inp["gate"])
+    zero_rows = (inp["gate"] == -20.0)
+    assert (qs[zero_rows] == 0).all(), "g = -20 zeroes the row"
+    _layer_case(cuda_lib, orc, inp, gated=True, report="gate extremes")
