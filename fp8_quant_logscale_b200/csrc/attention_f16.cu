@@ -401,26 +401,10 @@ __global__ void __launch_bounds__(kThreadsH, 1)
   }
 }
 
-typedef CUresult (*EncodeTiledFnH)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFnH encode_fn_h() {
-  static EncodeTiledFnH fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFnH>(ptr);
-  }
-  return fn;
-}
-
 // fp16 tensor map of rank `rank` (dims innermost first, strides in bytes for dims 1..rank-1).
 bool make_map_f16(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
                   const cuuint32_t* box) {
-  EncodeTiledFnH fn = encode_fn_h();
+  const TensorMapEncodeFn fn = tensor_map_encoder();
   if (!fn) return false;
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, rank, const_cast<void*>(base), dims, strides, box, estr,

@@ -7,6 +7,27 @@
 #include <stdint.h>
 
 namespace sdm {
+// cuTensorMapEncodeTiled, reached through the runtime's driver entry point (the
+// library does not link libcuda).  Looked up once per process; C++ makes the
+// initialisation of the local static thread-safe.  nullptr if unavailable.
+using TensorMapEncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                       const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                       CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                       CUtensorMapFloatOOBfill);
+inline TensorMapEncodeFn tensor_map_encoder() {
+  static const TensorMapEncodeFn fn = []() -> TensorMapEncodeFn {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<TensorMapEncodeFn>(ptr);
+    return nullptr;
+  }();
+  return fn;
+}
+}  // namespace sdm
+
+namespace sdm {
 
 constexpr int kHeadDim = 64;   // the only head dimension the kernels are built for
 constexpr int kKvTile = 128;   // keys per online-softmax block (one tcgen05 N=128 tile)

@@ -465,25 +465,9 @@ __global__ void __cluster_dims__(kClusterP, 1, 1) __launch_bounds__(kThreadsP, 1
   }
 }
 
-typedef CUresult (*EncodeTiledFnP)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFnP encode_fn_p() {
-  static EncodeTiledFnP fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFnP>(ptr);
-  }
-  return fn;
-}
-
 // bf16 [rows][heads][128] tensor, box {64, box_heads, box_rows}, 128-byte swizzle.
 bool make_map_rows(CUtensorMap* m, const void* base, int64_t rows, int heads, int box_heads, int box_rows) {
-  EncodeTiledFnP fn = encode_fn_p();
+  const TensorMapEncodeFn fn = tensor_map_encoder();
   if (!fn) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)kDP, (cuuint64_t)heads, (cuuint64_t)rows};
   const cuuint64_t strides[2] = {(cuuint64_t)kDP * 2, (cuuint64_t)heads * kDP * 2};
