@@ -65,10 +65,12 @@ __device__ __forceinline__ uint32_t o_col(int t) { return 128u * kTiles + 80u * 
 template <int kTiles>
 __device__ __forceinline__ uint32_t p_col(int t) { return 208u * kTiles + 32u * t; }
 
-// log2 of the largest probability a skipped tile may hold: e4m3 rounds
-// everything at or below 2^-10 to zero, so 2^-11 leaves room for the error of
-// the hardware 2^x and of the polynomial.
-constexpr float kDeadExponent = -11.0f;
+// log2 of the largest probability a skipped tile may hold. e4m3 rounds every
+// value at or below 2^-10 to zero (2^-10 is the midpoint between zero and the
+// smallest subnormal 2^-9, and the tie goes to the even code, zero). The 2^x
+// paths err by at most 3e-6 (polynomial) and 2^-22 (ex2.approx) relative, so
+// 2^-10.0625, 4% below 2^-10, keeps every skipped probability a zero code.
+constexpr float kDeadExponent = -10.0625f;
 
 constexpr long long kWaitLimit = 1LL << 31;   // ~1 s of SM clock: no legitimate wait comes close
 constexpr long long kDrainLimit = 1LL << 24;  // teardown waits for copies in flight
@@ -415,8 +417,8 @@ __global__ void __launch_bounds__(Cfg<kTiles>::kThreads, Cfg<kTiles>::kMinBlocks
       const float nm2 = -m2_new;
       // At or below 2^-10 every probability rounds to the e4m3 zero, through
       // ex2.approx and through the polynomial alike. fma is monotone in z
-      // (c2 > 0), so if the tile's largest logit lands below 2^-11 in every row
-      // of the warp, all of this warp's P_t is zero: skip the 2^x work and store
+      // (c2 > 0), so if the tile's largest logit lands below 2^kDeadExponent in
+      // every row of the warp, all of this warp's P_t is zero: skip the 2^x work and store
       // zeros, or nothing if the columns already hold zeros. The P V product
       // still runs and adds exact zeros, so the result is the same to the bit.
       // (Such a tile cannot raise the running max, so m_run and m2 stay.)

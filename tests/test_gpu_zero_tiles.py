@@ -40,7 +40,7 @@ def _hot_tile_inputs(N=2000, M=160, H=2, seed=21):
 def _dead_warp_tiles(orc, inp, split):
     """[H, row warps, key tiles] bool: every row of a 32-row warp has the tile's
     largest logit more than 11.5 log2 units below its running max (a margin over
-    the kernel's 11), computed in float64 from the oracle's FP8 codes; key tiles
+    the kernel's 10.0625), computed in float64 from the oracle's FP8 codes; key tiles
     restart their running max at every split-KV chunk boundary."""
     N = inp["N"]
     qs = orc.qscale(inp["q"], N, inp["c_h"])
