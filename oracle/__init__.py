@@ -85,7 +85,7 @@ def _declare(L):
     L.orc_quantize.argtypes = [_P, _I, _I64, _I, _I, _P, _P]
     L.orc_attention.restype = None
     L.orc_attention.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I64, _I64, _I,
-                                _P, _I64, _I64, _I64, _I, _D, _P, _P, _P]
+                                _P, _I64, _I64, _I64, _I, _I, _D, _P, _P, _P]
     L.orc_attention_exact.restype = None
     L.orc_attention_exact.argtypes = [_P, _P, _P, _I, _I, _I64, _I64, _I, _P, _I64, _P]
     L.orc_num_threads.restype = _I
@@ -176,12 +176,17 @@ def quantize(x: np.ndarray, scale: np.ndarray) -> np.ndarray:
     return out
 
 
+ARITH = {"definition": 0, "fp32": 1}
+
+
 def attention(q8, k8, v8, s_q, s_k, s_v, rows=None, bc: int = KV_TILE, split: int = 0,
-              quant_p: bool = True, delta: float = 0.0):
+              quant_p: bool = True, delta: float = 0.0, arith: str = "definition"):
     """FP8 online-softmax attention of the selected rows of q8 to all keys.
 
     q8 [B,H,T,d], k8/v8 [B,H,N,d] uint8 codes; s_* [B,H] fp32.
-    Returns (out16 [B,n,H,d] fp16, out [B,n,H,d] f64, allowance [B,n,H,d] f64).
+    arith: "definition" (the oracle: logits, exp and sums in double) or "fp32"
+    (a diagnostic: the single-precision sequence a tensor-core kernel takes).
+    Returns (out16 [B,n,H,d] fp16, out [B,n,H,d] f64, ambiguity report [B,n,H,d] f64).
     """
     q8 = np.ascontiguousarray(q8, np.uint8)
     k8 = np.ascontiguousarray(k8, np.uint8)
@@ -201,7 +206,7 @@ def attention(q8, k8, v8, s_q, s_k, s_v, rows=None, bc: int = KV_TILE, split: in
     allow = np.empty((B, n, H, d), np.float64)
     lib().orc_attention(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv),
                         B, H, T, N, d, _ptr(rows), n, int(bc), int(split),
-                        1 if quant_p else 0, float(delta),
+                        1 if quant_p else 0, ARITH[arith], float(delta),
                         _ptr(out16), _ptr(out), _ptr(allow))
     return out16.view(np.float16), out, allow
 

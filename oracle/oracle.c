@@ -245,41 +245,117 @@ static void e4m3_neighbours(uint8_t c, double* lo_mid, double* lo_alt,
 
 /*
  * One (b, h, query row) of the FP8 online-softmax attention over keys
- * [j_begin, j_end), in KV tiles of bc keys aligned to j_begin.
+ * [j_begin, j_end), in KV tiles of bc keys aligned to j_begin.  Two
+ * arithmetics, selected by `arith`:
  *
- * Logits and probabilities follow the kernel's single-precision arithmetic,
- * because the probability's e4m3 code is an integer decided by floating point:
- *   z_j  = sum_e q8[e] * k8_j[e]           fp32, e ascending (products exact)
- *   c2   = fp32(fp32(s_q*s_k) * fp32(log2(e)/sqrt(d)))
- *   m    = running max of z over the keys seen so far, m2 = fp32(m * c2)
- *   t_j  = fma(z_j, c2, -m2)               fp32, one rounding
- *   p_j  = fp32(2^t_j)                     exp2 correctly rounded to fp32
- *   P8_j = e4m3(p_j)                       unit scale, p_j <= ~1
- * Whenever a tile raises m, the running sums are rescaled by
+ * ORC_ARITH_DEFINITION (the oracle proper) -- the layer's definition written
+ * out in double ([FP8] opening section: logits of the e4m3 Q and K with the
+ * per-head scales, online softmax over key tiles, P quantised to e4m3 before
+ * P.V; the softmax scale is SDPA's default 1/sqrt(d)):
+ *   z_j  = sum_e dec(q8[e]) * dec(k8_j[e])    exact: every product is a multiple
+ *                                             of 2^-18 below 2^18, so 64 of them
+ *                                             add up within double's 53 bits
+ *   x_j  = z_j * (s_q * s_k / sqrt(d))        natural-log units
+ *   per tile: m' = max(m, max_j x_j),  P_j = exp(x_j - m'),  P8_j = e4m3(P_j)
+ *   when m' > m:  l and acc are multiplied by alpha = exp(m - m')
+ *   l += sum_j dec(P8_j);   acc += sum_j dec(P8_j) * dec(v8_j)
+ *
+ * ORC_ARITH_FP32 (a diagnostic only) -- the same steps in the single-precision
+ * sequence a tensor-core kernel takes, in base-2 units:
+ *   z_j  = fp32 sum, e ascending;   c2 = fp32(fp32(s_q*s_k) * fp32(log2(e)/sqrt(d)))
+ *   m2 = fp32(m * c2);  t_j = fma(z_j, c2, -m2);  p_j = fp32(2^t_j);  P8_j = e4m3(p_j)
  *   alpha = 2^(fp32(m2_old - m2_new)).
- * Sums run in double:  l = sum alpha-weighted dec(P8);  acc = sum dec(P8)*dec(v8).
- * (With quant_p == 0 the e4m3 rounding of p is skipped: the plain softmax.)
+ * It shows how far an fp32 implementation's e4m3 codes move from the
+ * definition's; no test gates the CUDA path against it.
  *
- * The partial result is (m2, l, acc[d]).  For the ambiguity allowance, keys
- * whose p_j lies within relative distance delta of an e4m3 rounding midpoint
- * are ones where a correct implementation may legitimately pick the other
- * code; amb0 accumulates the weight change that choice would make and
- * amb1[e] that change times |dec(v8_j[e])|, with the same rescaling as l/acc.
+ * In both, the running maximum is reported in base-2 units (m2 = m * log2 e
+ * for the definition), and with quant_p == 0 the e4m3 rounding of P is
+ * skipped: the plain softmax.
+ *
+ * Ambiguity report: keys whose probability lies within relative distance
+ * delta of an e4m3 rounding midpoint are ones where an implementation whose
+ * probabilities err by that much may pick the other code; amb0 accumulates the
+ * weight change that choice would make and amb1[e] that change times
+ * |dec(v8_j[e])|, with the same rescaling as l/acc.
  */
+enum { ORC_ARITH_DEFINITION = 0, ORC_ARITH_FP32 = 1 };
+
 typedef struct {
-    float m2;      /* running max in log2 units; -inf if no key */
+    double m2;     /* running max in log2 units; -inf if no key */
     double l, amb0;
     double* acc;   /* [d] */
     double* amb1;  /* [d] */
 } orc_partial;
 
-static void attend_range(const uint8_t* q8row, const uint8_t* k8, const uint8_t* v8,
-                         int64_t j_begin, int64_t j_end, int d, float c2,
-                         int64_t bc, int quant_p, double delta, orc_partial* st,
-                         float* zbuf) {
-    float m = -INFINITY;                      /* running max of z (raw units) */
+static void partial_scale(orc_partial* st, int d, double alpha) {
+    st->l *= alpha; st->amb0 *= alpha;
+    for (int e = 0; e < d; ++e) { st->acc[e] *= alpha; st->amb1[e] *= alpha; }
+}
+
+/* Adds key j with probability p (>= 0) to the running sums: its e4m3 weight
+ * (or p itself when quant_p == 0) and its ambiguity contribution. */
+static void partial_add_key(orc_partial* st, double p, const uint8_t* vj, int d,
+                            int quant_p, double delta) {
+    double w = p, dw = 0.0;
+    if (quant_p) {
+        uint8_t c = orc_e4m3_encode(p);
+        w = orc_e4m3_decode(c);
+        if (p > 0.0 && delta > 0.0) {
+            double lo_mid, lo_alt, hi_mid, hi_alt;
+            e4m3_neighbours(c, &lo_mid, &lo_alt, &hi_mid, &hi_alt);
+            if (fabs(p - lo_mid) <= delta * p) dw = fabs(w - lo_alt);
+            if (fabs(p - hi_mid) <= delta * p) dw = fabs(hi_alt - w);
+        }
+    }
+    if (w == 0.0 && dw == 0.0) return;
+    st->l += w; st->amb0 += dw;
+    for (int e = 0; e < d; ++e) {
+        double ve = g_e4m3[vj[e]];
+        st->acc[e] += w * ve;
+        st->amb1[e] += dw * fabs(ve);
+    }
+}
+
+static void partial_reset(orc_partial* st, int d) {
     st->m2 = -INFINITY; st->l = 0; st->amb0 = 0;
     for (int e = 0; e < d; ++e) { st->acc[e] = 0; st->amb1[e] = 0; }
+}
+
+static const double kLog2e = 1.4426950408889634074;
+
+static void attend_range_definition(const uint8_t* q8row, const uint8_t* k8, const uint8_t* v8,
+                                    int64_t j_begin, int64_t j_end, int d, double scale,
+                                    int64_t bc, int quant_p, double delta, orc_partial* st,
+                                    double* xbuf) {
+    double m = -INFINITY;                     /* running max of x (natural-log units) */
+    partial_reset(st, d);
+    for (int64_t j0 = j_begin; j0 < j_end; j0 += bc) {
+        int64_t j1 = j0 + bc < j_end ? j0 + bc : j_end;
+        double mt = m;
+        for (int64_t j = j0; j < j1; ++j) {
+            const uint8_t* kj = k8 + j * d;
+            double z = 0.0;
+            for (int e = 0; e < d; ++e) z += g_e4m3[q8row[e]] * g_e4m3[kj[e]];
+            xbuf[j - j0] = z * scale;
+            if (xbuf[j - j0] > mt) mt = xbuf[j - j0];
+        }
+        if (mt > m) {
+            partial_scale(st, d, m == -INFINITY ? 0.0 : exp(m - mt));
+            m = mt;
+        }
+        for (int64_t j = j0; j < j1; ++j)
+            partial_add_key(st, exp(xbuf[j - j0] - m), v8 + j * d, d, quant_p, delta);
+    }
+    st->m2 = m * kLog2e;
+}
+
+static void attend_range_f32(const uint8_t* q8row, const uint8_t* k8, const uint8_t* v8,
+                             int64_t j_begin, int64_t j_end, int d, float c2,
+                             int64_t bc, int quant_p, double delta, orc_partial* st,
+                             double* xbuf) {
+    float m = -INFINITY;                      /* running max of z (raw units) */
+    float m2 = -INFINITY;
+    partial_reset(st, d);
     for (int64_t j0 = j_begin; j0 < j_end; j0 += bc) {
         int64_t j1 = j0 + bc < j_end ? j0 + bc : j_end;
         float mt = m;
@@ -287,46 +363,25 @@ static void attend_range(const uint8_t* q8row, const uint8_t* k8, const uint8_t*
             const uint8_t* kj = k8 + j * d;
             float z = 0.0f;   /* each product of two e4m3 values is exact in fp32 */
             for (int e = 0; e < d; ++e) z += g_e4m3_f[q8row[e]] * g_e4m3_f[kj[e]];
-            zbuf[j - j0] = z;
+            xbuf[j - j0] = z;
             if (z > mt) mt = z;
         }
         float m2_new = mt * c2;
         if (mt > m) {
-            double alpha = (m == -INFINITY) ? 0.0 : exp2((double)(st->m2 - m2_new));
-            st->l *= alpha; st->amb0 *= alpha;
-            for (int e = 0; e < d; ++e) { st->acc[e] *= alpha; st->amb1[e] *= alpha; }
-            m = mt; st->m2 = m2_new;
+            partial_scale(st, d, m == -INFINITY ? 0.0 : exp2((double)(m2 - m2_new)));
+            m = mt; m2 = m2_new;
         }
         for (int64_t j = j0; j < j1; ++j) {
-            float t = fmaf(zbuf[j - j0], c2, -st->m2);
-            float p = (float)exp2((double)t);
-            double w = p;
-            double dw = 0.0;                  /* weight change of the other code */
-            if (quant_p) {
-                uint8_t c = orc_e4m3_encode((double)p);
-                w = orc_e4m3_decode(c);
-                if (p > 0.0f && delta > 0.0) {
-                    double lo_mid, lo_alt, hi_mid, hi_alt;
-                    e4m3_neighbours(c, &lo_mid, &lo_alt, &hi_mid, &hi_alt);
-                    if (fabs((double)p - lo_mid) <= delta * p) dw = fabs(w - lo_alt);
-                    if (fabs((double)p - hi_mid) <= delta * p) dw = fabs(hi_alt - w);
-                }
-            }
-            if (w == 0.0 && dw == 0.0) continue;
-            const uint8_t* vj = v8 + j * d;
-            st->l += w; st->amb0 += dw;
-            for (int e = 0; e < d; ++e) {
-                double ve = g_e4m3[vj[e]];
-                st->acc[e] += w * ve;
-                st->amb1[e] += dw * fabs(ve);
-            }
+            float t = fmaf((float)xbuf[j - j0], c2, -m2);
+            partial_add_key(st, (double)(float)exp2((double)t), v8 + j * d, d, quant_p, delta);
         }
     }
+    st->m2 = m2;
 }
 
 static float softmax_c2(float s_q, float s_k, int d) {
     float sqk = s_q * s_k;
-    float k2 = (float)(1.4426950408889634074 / sqrt((double)d)); /* log2(e)/sqrt(d) */
+    float k2 = (float)(kLog2e / sqrt((double)d)); /* log2(e)/sqrt(d) */
     return sqk * k2;
 }
 
@@ -339,13 +394,15 @@ static float softmax_c2(float s_q, float s_k, int d) {
  *                      >0: cached prediction ([FP8] "model.predict(queries)"
  *                      after fit) -- keys cut into chunks of `split` keys,
  *                      each processed from a fresh state, then combined in
- *                      chunk order:  M2 = max m2_s;  w_s = 2^(m2_s - M2);
- *                      L = sum w_s l_s;  ACC = sum w_s acc_s.
+ *                      chunk order:  M = max m_s;  w_s = exp(m_s - M);
+ *                      L = sum w_s l_s;  ACC = sum w_s acc_s  (in base-2 units
+ *                      and fp32 exponent differences under ORC_ARITH_FP32).
+ *   arith              ORC_ARITH_DEFINITION or ORC_ARITH_FP32 (see above)
  *   out16 [B][n_rows][H][d]   fp16 bits of ACC * s_v / L
  *   out   [B][n_rows][H][d]   the same value before fp16 rounding (double)
- *   allow [B][n_rows][H][d]   ambiguity allowance (may be NULL): first-order
- *                      bound on |O| change if every key whose p sits within
- *                      relative delta of an e4m3 midpoint took the other code:
+ *   allow [B][n_rows][H][d]   ambiguity report (may be NULL): first-order
+ *                      change of O if every key whose p sits within relative
+ *                      delta of an e4m3 midpoint took the other code:
  *                      s_v * (amb1[e] + amb0 * vmax_e) / L, where vmax_e is the
  *                      largest |dec(v8[.][e])| of the head.
  */
@@ -353,7 +410,7 @@ void orc_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
                    const float* s_q, const float* s_k, const float* s_v,
                    int B, int H, int64_t T, int64_t N, int d,
                    const int64_t* rows, int64_t n_rows, int64_t bc, int64_t split,
-                   int quant_p, double delta,
+                   int quant_p, int arith, double delta,
                    uint16_t* out16, double* out, double* allow) {
     int64_t n_chunks = (split > 0) ? (N + split - 1) / split : 1;
     int64_t chunk = (split > 0) ? split : N;
@@ -367,7 +424,7 @@ void orc_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
             }
     #pragma omp parallel
     {
-        float* zbuf = (float*)malloc(sizeof(float) * (size_t)bc);
+        double* xbuf = (double*)malloc(sizeof(double) * (size_t)bc);
         double* tmp = (double*)malloc(sizeof(double) * (size_t)(4 * d));
         orc_partial st; st.acc = tmp; st.amb1 = tmp + d;
         double* ACC = tmp + 2 * d; double* A1 = tmp + 3 * d;
@@ -378,22 +435,32 @@ void orc_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
             const uint8_t* qrow = q8 + (bh * T + i) * d;
             const uint8_t* kb = k8 + bh * N * d;
             const uint8_t* vb = v8 + bh * N * d;
+            /* softmax scale of the definition: s_q * s_k / sqrt(d), in double */
+            double scale = (double)s_q[bh] * (double)s_k[bh] / sqrt((double)d);
             float c2 = softmax_c2(s_q[bh], s_k[bh], d);
-            float M2 = -INFINITY;
+            double M = -INFINITY;             /* natural-log units (definition) or base 2 */
             double L = 0, A0 = 0;
             for (int e = 0; e < d; ++e) { ACC[e] = 0; A1[e] = 0; }
             /* chunk maxima first, then the fixed-order combine */
             for (int64_t s = 0; s < n_chunks; ++s) {
                 int64_t jb = s * chunk, je = jb + chunk < N ? jb + chunk : N;
-                attend_range(qrow, kb, vb, jb, je, d, c2, bc, quant_p, delta, &st, zbuf);
+                double ms;
+                if (arith == ORC_ARITH_FP32) {
+                    attend_range_f32(qrow, kb, vb, jb, je, d, c2, bc, quant_p, delta, &st, xbuf);
+                    ms = st.m2;
+                } else {
+                    attend_range_definition(qrow, kb, vb, jb, je, d, scale, bc, quant_p, delta, &st, xbuf);
+                    ms = st.m2 / kLog2e;      /* back to natural-log units */
+                }
                 if (st.m2 == -INFINITY) continue;
-                if (st.m2 > M2) {
-                    double a = (M2 == -INFINITY) ? 0.0 : exp2((double)(M2 - st.m2));
+                if (ms > M) {
+                    double a = (M == -INFINITY) ? 0.0
+                             : (arith == ORC_ARITH_FP32) ? exp2((double)(float)(M - ms)) : exp(M - ms);
                     L *= a; A0 *= a;
                     for (int e = 0; e < d; ++e) { ACC[e] *= a; A1[e] *= a; }
-                    M2 = st.m2;
+                    M = ms;
                 }
-                double w = exp2((double)(st.m2 - M2));
+                double w = (arith == ORC_ARITH_FP32) ? exp2((double)(float)(ms - M)) : exp(ms - M);
                 L += w * st.l; A0 += w * st.amb0;
                 for (int e = 0; e < d; ++e) { ACC[e] += w * st.acc[e]; A1[e] += w * st.amb1[e]; }
             }
@@ -405,7 +472,7 @@ void orc_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
                 if (allow) allow[o + e] = (double)s_v[bh] * (A1[e] + A0 * vmax[bh * d + e]) / L;
             }
         }
-        free(zbuf); free(tmp);
+        free(xbuf); free(tmp);
     }
     free(vmax);
 }

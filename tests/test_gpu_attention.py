@@ -1,10 +1,11 @@
 """GPU parity of steps 1-3 (one call of the FP8 ICL attention layer) against the oracle.
 
-FP8 tensors and scales are compared bit for bit; attention outputs within the
-specification's gates (max |d| 2e-2, mean |d| 1e-3), where the oracle adds an
-allowance only for keys whose probability sits within relative 1e-4 of an
-e4m3 rounding midpoint (either code is a correct result there).  The error
-against exact attention is printed for the record.
+FP8 tensors and scales are compared bit for bit; attention outputs against the
+oracle's double-precision definition within the specification's gates: every
+element within max(2e-2, one fp16 ulp of its value) and mean |d| <= 1e-3, with
+nothing added for keys whose probability sits next to an e4m3 rounding midpoint
+(the share of such outputs is only reported).  The error against exact
+attention is printed for the record.
 """
 import os
 
@@ -65,9 +66,10 @@ def _layer_case(cuda_lib, orc, inp, gated=False, rows=None, report=""):
     stats = gate(got, o, allow, report)
     # error against exact attention, reported only: on at most 256 of the checked rows
     # (the double-precision reference is the slowest part of the large cases)
-    sub = slice(None) if rows is None or len(rows) <= 256 else slice(None, None, -(-len(rows) // 256))
-    exact = orc.attention_exact(qs, inp["k"], inp["v"], rows=None if rows is None else rows[sub])
-    e = (got if rows is None else got[:, sub]).astype(np.float64) - exact
+    sel = np.arange(N + M) if rows is None else rows
+    pos = np.arange(sel.size)[::-(-sel.size // 256)]
+    exact = orc.attention_exact(qs, inp["k"], inp["v"], rows=sel[pos])
+    e = got[:, pos].astype(np.float64) - exact
     stats["vs_exact_rel_rms"] = float(np.sqrt((e ** 2).mean() / (exact ** 2).mean()))
     print(f"\n{report}: {stats}")
     return stats
@@ -92,16 +94,18 @@ def _sample_rows(N, M, n_ctx_rows, n_q_rows, seed):
     return np.sort(np.concatenate([ctx, qry])).astype(np.int64)
 
 
-def test_layer_16k_sampled(cuda_lib, orc):
-    w = WORKLOADS["icl_n16k_m1k_h8"]
-    inp = make_inputs(w)
-    _layer_case(cuda_lib, orc, inp, rows=_sample_rows(w.n_ctx, w.n_query, 256, 256, 2), report="16K")
+def test_layer_16k_every_row(cuda_lib, orc):
+    """The 16K workload (per-head U(0.5, 4) factors): every context and query row."""
+    inp = make_inputs(WORKLOADS["icl_n16k_m1k_h8"])
+    _layer_case(cuda_lib, orc, inp, report="16K every row")
 
 
 def test_layer_128k_gated_sampled(cuda_lib, orc):
+    """The 128K gated workload with x20 outliers: a seeded sample of 256 context rows
+    and every query row."""
     w = WORKLOADS["icl_n128k_m1k_h8_gated"]
     inp = make_inputs(w)
-    _layer_case(cuda_lib, orc, inp, gated=True, rows=_sample_rows(w.n_ctx, w.n_query, 128, 128, 3),
+    _layer_case(cuda_lib, orc, inp, gated=True, rows=_sample_rows(w.n_ctx, w.n_query, 256, w.n_query, 3),
                 report="128K gated")
 
 

@@ -2,7 +2,9 @@
 (sdm_cached_attention_offload): chunk by chunk through two device staging slots,
 it must give the same bits as sdm_cached_attention on the device-resident cache
 (the same split-KV chunks, the same fixed-order combine), with and without a
-separate copy stream, for uniform and ragged caches, and at full size."""
+separate copy stream, for uniform and ragged caches, and at full size -- and,
+on its own, match the oracle's chunked attention within the layer's gates (a
+seeded sample of queries at full size, every query of a ragged cache)."""
 import ctypes
 
 import numpy as np
@@ -10,7 +12,7 @@ import pytest
 import torch
 
 from fp8_quant_logscale_b200.workloads import WORKLOADS, make_inputs
-from parity import dev, host
+from parity import DELTA, dev, gate, host
 
 pytestmark = pytest.mark.gpu
 
@@ -59,16 +61,30 @@ def test_offload_gated_queries(cuda_lib):
                 cuda_lib.cached_attention(q, cache, c_h, gate=g))
 
 
-def test_offload_ragged_cache(cuda_lib):
+def test_offload_ragged_cache(cuda_lib, orc):
     H, B, N, M = 2, 3, 3000, 40
-    inp, cache = fitted(cuda_lib, N, H, B=B, ctx_len=[900, 3000, 1025], wname="ragged_b16_n16k_m1k_h8")
+    lens = [900, 3000, 1025]
+    inp, cache = fitted(cuda_lib, N, H, B=B, ctx_len=lens, wname="ragged_b16_n16k_m1k_h8")
     off = cache.offload()
-    q, c_h = dev(queries(H, M, B)), dev(inp["c_h"])
-    assert same(cuda_lib.cached_attention_offload(q, off, c_h), cuda_lib.cached_attention(q, cache, c_h))
+    qn = queries(H, M, B)
+    q, c_h = dev(qn), dev(inp["c_h"])
+    got = cuda_lib.cached_attention_offload(q, off, c_h)
+    assert same(got, cuda_lib.cached_attention(q, cache, c_h))
+    # against the oracle: estimator b is the layer on its own n_b context rows
+    got = host(got)
+    r = orc.layer_ragged(inp["q"], inp["k"], inp["v"], lens, inp["c_h"])
+    for b, n in enumerate(lens):
+        q8 = orc.quantize(orc.qscale(qn[b:b + 1], n, inp["c_h"]), r["s_q"][b:b + 1])
+        _, o, allow = orc.attention(q8, np.ascontiguousarray(r["k8"][b:b + 1, :, :n]),
+                                    np.ascontiguousarray(r["v8"][b:b + 1, :, :n]), r["s_q"][b:b + 1],
+                                    r["s_k"][b:b + 1], r["s_v"][b:b + 1], split=orc.split_keys(N), delta=DELTA)
+        print(f"\noffload ragged batch {b} n_b={n}:", gate(got[b:b + 1], o, allow, f"offload ragged b{b}"))
 
 
-def test_offload_full_size(cuda_lib):
-    """The 524,288-key cache (537 MB of K8 / V8^T in host memory), 1,024 queries."""
+def test_offload_full_size(cuda_lib, orc):
+    """The 524,288-key cache (537 MB of K8 / V8^T in host memory), 1,024 queries: equal to
+    the resident cache bit for bit, and a seeded sample of 256 queries (every head)
+    against the oracle's chunked attention."""
     w = WORKLOADS["cached_n512k_m1k_h8"]
     inp = make_inputs(w)
     N, M, H = w.n_ctx, w.n_query, w.heads
@@ -79,8 +95,16 @@ def test_offload_full_size(cuda_lib):
     off = cache.offload()
     del cache
     torch.cuda.empty_cache()
-    assert same(cuda_lib.cached_attention_offload(q, off, c_h), want)
+    got = cuda_lib.cached_attention_offload(q, off, c_h)
+    assert same(got, want)
     assert same(cuda_lib.cached_attention_offload(q[:, :1].contiguous(), off, c_h), want[:, :1])
+    rows = np.sort(np.random.default_rng(5).choice(M, 256, replace=False)).astype(np.int64)
+    qs = orc.qscale(inp["q"], N, inp["c_h"])
+    s_q, s_k, s_v = (orc.context_scales(x, N) for x in (qs, inp["k"], inp["v"]))
+    q8 = orc.quantize(orc.qscale(inp["queries"], N, inp["c_h"]), s_q)
+    _, o, allow = orc.attention(q8, orc.quantize(inp["k"], s_k), orc.quantize(inp["v"], s_v), s_q, s_k, s_v,
+                                rows=rows, split=orc.split_keys(N), delta=DELTA)
+    print("\noffload 512K, 256 queries:", gate(host(got)[:, rows], o, allow, "offload 512K"))
 
 
 def test_offload_rejects_pageable_memory(cuda_lib):

@@ -1,12 +1,15 @@
 """Pins of the oracle's FP8 attention and cached (split-KV) prediction (CPU only).
 
-Against: a naive full-row double softmax (quantisation of P switched off), a
-materialised-P implementation in numpy + torch's e4m3 cast, a hand-worked
-golden example with exact powers of two, Q = 0 (mean of V), constant V (the
-row sum normalises), permutation of the context rows, partitions of the query
-batch for the cached path, and the pages' block-level accuracy bound against
-exact attention ("[FP8 4/5]" KumoTabular page, review of
-test/models/test_attention_quantization.py: relative RMS < 0.08).
+The oracle's attention is the layer's definition in double precision (logits of
+the e4m3 Q and K times s_q s_k / sqrt(d), online softmax over 128-key tiles, P
+rounded to e4m3 against the running maximum before P.V).  It is pinned against:
+a naive full-row double softmax (quantisation of P switched off); a
+materialised-P restatement in numpy with torch's e4m3 decode and an e4m3
+rounding written here, over several tile sizes and split-KV chunkings; a
+hand-worked golden example with exact powers of two; Q = 0 (mean of V);
+constant V (the row sum normalises); permutation of the context rows; and
+partitions of the query batch for the cached path.  The single-precision
+diagnostic arithmetic is pinned by its own materialised version.
 """
 import os
 
@@ -81,10 +84,22 @@ def test_golden_worked_example(orc):
     k8 = np.stack([np.full(64, c, np.uint8) for c in (0x00, 0x08, 0x10)])[None, None]
     v8 = np.stack([np.full(64, c, np.uint8) for c in (0x38, 0x40, 0x48)])[None, None]
     one = np.ones((1, 1), np.float32)
+    want = float(lines["out"][0])
+    # in the definition the logit of key j is z_j * s_k / 8 = z_j * ln2 * (1 + eps), with eps the
+    # distance of the fp32 s_k from 8 / log2(e): the probabilities 2^(-2(1+eps)), 2^(-(1+eps)), 1
+    # still round to the e4m3 values 1/4, 1/2, 1, but a running-sum rescale exp(m - m') is 1/2 or
+    # 1/4 only to within 2 ln2 |eps| relative
+    eps = abs(float(sk) * LOG2E / 8.0 - 1.0)
+    assert eps < 2.0 ** -22
     for bc in (1, 2, 128):
+        # with every key in one tile O is exactly 3; with smaller tiles within the rescale error
         o16, o, _ = orc.attention(q8, k8, v8, one, np.full((1, 1), sk, np.float32), one, bc=bc)
-        assert (o == float(lines["out"][0])).all(), (bc, o[0, 0, 0, :4])
+        tol = 0.0 if bc >= 3 else 4.0 * np.log(2.0) * eps * want
+        assert (np.abs(o - want) <= tol).all(), (bc, o[0, 0, 0, :4])
         assert (o16.astype(np.float64) == 3.0).all()
+        # the single-precision diagnostic arithmetic lands on the same powers of two exactly
+        o16, o, _ = orc.attention(q8, k8, v8, one, np.full((1, 1), sk, np.float32), one, bc=bc, arith="fp32")
+        assert (o == want).all(), (bc, o[0, 0, 0, :4])
 
 
 @pytest.mark.parametrize("bc", [7, 128])
@@ -106,8 +121,64 @@ def test_constant_v_normalises_to_one(orc):
     assert (o16.astype(np.float64) == 1.0).all()
 
 
-def test_materialised_p_matches_online(orc):
-    """Full P matrix in numpy (fp32 logits in e order, torch e4m3 cast) vs the online oracle with one tile."""
+def _e4m3_round(p):
+    """Nearest e4m3 value of p >= 0 (ties to even), for p <= 448: binade spacing
+    2^(e-3), subnormal spacing 2^-9.  Written here from the format, independent of
+    the oracle's codec."""
+    p = np.asarray(p, np.float64)
+    _, e = np.frexp(p)                       # p in [2^(e-1), 2^e)
+    step = np.exp2(np.maximum(e - 1, -6) - 3)
+    return np.rint(p / step) * step          # p / step is exact; rint ties to even
+
+
+def _torch_e4m3_decode(codes):
+    return torch.from_numpy(np.ascontiguousarray(codes)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def _materialised_definition(q8, k8, v8, sq, sk, sv, bc, split=0):
+    """The whole P matrix at once: x = z s_q s_k / 8 with z exact, the running maximum
+    at each key's tile (restarting at every split chunk), P8 = e4m3(exp(x - run)),
+    each key weighted by exp(run - M) against the row's overall maximum M."""
+    q, k, v = (_torch_e4m3_decode(c) for c in (q8, k8, v8))     # [B,H,*,d]
+    B, H, T, _ = q.shape
+    N = k.shape[2]
+    x = (q @ k.transpose(0, 1, 3, 2)) * (sq.astype(np.float64) * sk.astype(np.float64) / 8.0)[..., None, None]
+    chunk = split if split > 0 else N
+    run = np.empty_like(x)
+    for c0 in range(0, N, chunk):
+        m = np.full(x.shape[:-1], -np.inf)
+        for j0 in range(c0, min(N, c0 + chunk), bc):
+            j1 = min(j0 + bc, c0 + chunk, N)
+            m = np.maximum(m, x[..., j0:j1].max(-1))
+            run[..., j0:j1] = m[..., None]
+    M = x.max(-1, keepdims=True)
+    w = _e4m3_round(np.exp(x - run)) * np.exp(run - M)
+    o = (w @ v) / w.sum(-1, keepdims=True) * sv[..., None, None]
+    return o.transpose(0, 2, 1, 3)
+
+
+@pytest.mark.parametrize("bc,split", [(200, 0), (128, 0), (7, 0), (32, 96), (128, 128)])
+def test_materialised_p_matches_online(orc, bc, split):
+    """The online oracle (tile by tile, rescaling at every new maximum, chunks combined
+    in order) against the materialised restatement: the same e4m3 codes, sums equal to
+    double rounding."""
+    q8, k8, v8, sq, sk, sv = _problem(orc, T=24, N=200, seed=7, qscale=1.0)
+    want = _materialised_definition(q8, k8, v8, sq, sk, sv, bc, split)
+    _, out, _ = orc.attention(q8, k8, v8, sq, sk, sv, bc=bc, split=split)
+    assert np.abs(out - want).max() <= 1e-12 * np.abs(want).max()
+
+
+def test_materialised_p_finds_a_tile_error(orc):
+    """The materialised restatement tells tile sizes apart on these inputs, so the pin
+    above would catch a wrong tile boundary or a missed rescale."""
+    q8, k8, v8, sq, sk, sv = _problem(orc, T=24, N=200, seed=7, qscale=1.0)
+    a = _materialised_definition(q8, k8, v8, sq, sk, sv, 128)
+    b = _materialised_definition(q8, k8, v8, sq, sk, sv, 7)
+    assert np.abs(a - b).max() > 1e-6
+
+
+def test_materialised_p_matches_online_fp32_diagnostic(orc):
+    """The single-precision diagnostic: fp32 logits in e order, torch's e4m3 cast, one tile."""
     q8, k8, v8, sq, sk, sv = _problem(orc, T=24, N=200, seed=7, qscale=1.0)
     qf = orc.e4m3_decode(q8).astype(np.float32)
     kf = orc.e4m3_decode(k8).astype(np.float32)
@@ -121,8 +192,18 @@ def test_materialised_p_matches_online(orc):
     p8 = orc.e4m3_decode(torch.from_numpy(p).to(torch.float8_e4m3fn).view(torch.uint8).numpy())
     vf = orc.e4m3_decode(v8)
     want = (np.einsum("bhtn,bhnd->bhtd", p8, vf) / p8.sum(-1)[..., None] * sv[..., None, None]).transpose(0, 2, 1, 3)
-    _, out, allow = orc.attention(q8, k8, v8, sq, sk, sv, bc=200, delta=1e-6)
+    _, out, allow = orc.attention(q8, k8, v8, sq, sk, sv, bc=200, delta=1e-6, arith="fp32")
     assert (np.abs(out - want) <= 1e-12 + allow).all()
+
+
+def test_definition_and_fp32_arithmetic_agree_closely(orc):
+    """The definition and the single-precision sequence give nearly the same outputs:
+    their e4m3 probability codes differ only where a probability sits next to a
+    rounding midpoint, and the rescale factors by fp32 rounding (relative 1e-6 here)."""
+    q8, k8, v8, sq, sk, sv = _problem(orc, T=40, N=300, seed=29, qscale=1.0)
+    _, a, allow = orc.attention(q8, k8, v8, sq, sk, sv, delta=1e-5)
+    _, b, _ = orc.attention(q8, k8, v8, sq, sk, sv, arith="fp32")
+    assert (np.abs(a - b) <= 1e-6 * np.abs(a).max() + allow).all()
 
 
 def test_context_permutation(orc):

@@ -3,10 +3,11 @@
 It serves callers that cannot allocate device memory for the library (paths
 that must not call cudaMalloc, plugins whose framework owns all device memory):
 its amax scratch is a fixed array inside the library.  Its results must equal
-those of sdm_fp8_quantize_context bit for bit (FP8 codes and scales are
-compared exactly, as everywhere else), on two calls in a row -- the second
-with a smaller amax than the first, so stale scratch would show -- and sizes
-past the array's limit must be refused before any work is enqueued.
+those of sdm_fp8_quantize_context and the oracle's context scales and e4m3
+codes bit for bit (FP8 codes and scales are compared exactly, as everywhere
+else), on two calls in a row -- the second with a smaller amax than the first,
+so stale scratch would show -- and sizes past the array's limit must be
+refused before any work is enqueued.
 This file is collected last on purpose."""
 import ctypes
 
@@ -37,7 +38,7 @@ def _noalloc_call(L, q, k, v, N):
     return q8, cache
 
 
-def test_noalloc_matches_workspace_entry_point_twice(cuda_lib):
+def test_noalloc_matches_workspace_entry_point_twice(cuda_lib, orc):
     L = binding.lib()
     N = 1000
     for scale in (4.0, 0.5):          # second call: smaller amax than the first
@@ -50,6 +51,14 @@ def test_noalloc_matches_workspace_entry_point_twice(cuda_lib):
         assert torch.equal(q8, q8_ref)
         assert torch.equal(c.k8, c_ref.k8)
         assert torch.equal(c.v8t, c_ref.v8t)
+        # and against the oracle: context-only scales, then the e4m3 codes
+        qn, kn, vn = (x.cpu().numpy() for x in (q, k, v))
+        s_q, s_k, s_v = (orc.context_scales(x, N) for x in (qn, kn, vn))
+        sc = c.scales.cpu().numpy()
+        assert (sc[0] == s_q).all() and (sc[1] == s_k).all() and (sc[2] == s_v).all()
+        assert (q8.cpu().numpy() == orc.quantize(qn, s_q)).all()
+        assert (c.k8.cpu().numpy() == orc.quantize(kn, s_k)).all()
+        assert (c.v8t.cpu().numpy()[..., :N] == orc.quantize(vn, s_v).transpose(0, 1, 3, 2)).all()
 
 
 def test_noalloc_rejects_sizes_past_its_array(cuda_lib):
