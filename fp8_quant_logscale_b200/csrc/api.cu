@@ -821,23 +821,56 @@ static __device__ __align__(256) uint32_t g_noalloc_amax[3 * kNoAllocMaxBatchHea
 
 // In host code `g_noalloc_amax` names a host-side stand-in, not device memory,
 // so kernels must be given the address the runtime reports for it -- looked up
-// once per device, with that device current.
+// with the device current, once per device and CUDA context: the address is
+// taken again when the device's current context is not the one it was taken in
+// (after cudaDeviceReset, or a primary context released and created anew), so
+// no call uses an address of a context that is gone.
 constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mu;
-uint32_t* g_noalloc_addr[kNoAllocMaxDevices] = {};
+struct NoAllocSlot {
+  CUcontext ctx;
+  uint32_t* addr;
+};
+NoAllocSlot g_noalloc_slot[kNoAllocMaxDevices] = {};
+
+// cuCtxGetCurrent through the runtime's driver entry point (the library does
+// not link libcuda); looked up once per process.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current() {
+  static const CtxGetCurrentFn fn = []() -> CtxGetCurrentFn {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<CtxGetCurrentFn>(ptr);
+    return nullptr;
+  }();
+  return fn;
+}
 
 sdm_status noalloc_scratch(int dev, uint32_t** out) {
   if (dev < 0 || dev >= kNoAllocMaxDevices) return SDM_ERR_UNSUPPORTED;
+  const CtxGetCurrentFn get_ctx = ctx_get_current();
+  CUcontext ctx = nullptr;  // null if no runtime call has made the primary context current yet
+  if (get_ctx == nullptr || get_ctx(&ctx) != CUDA_SUCCESS) return SDM_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_addr[dev] == nullptr) {
+  NoAllocSlot& slot = g_noalloc_slot[dev];
+  if (slot.addr == nullptr || ctx == nullptr || slot.ctx != ctx) {
     void* p = nullptr;
+    // also makes the device's primary context current if it was not yet
     if (cudaGetSymbolAddress(&p, g_noalloc_amax) != cudaSuccess || p == nullptr) {
       cudaGetLastError();
+      slot.addr = nullptr;
       return SDM_ERR_CUDA;
     }
-    g_noalloc_addr[dev] = static_cast<uint32_t*>(p);
+    if (ctx == nullptr && (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr)) {
+      slot.addr = nullptr;
+      return SDM_ERR_CUDA;
+    }
+    slot.ctx = ctx;
+    slot.addr = static_cast<uint32_t*>(p);
   }
-  *out = g_noalloc_addr[dev];
+  *out = slot.addr;
   return SDM_OK;
 }
 

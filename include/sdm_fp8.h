@@ -334,7 +334,9 @@ sdm_status sdm_gqa_prefill(const void* q, const void* k, const void* v, const in
  *     every GPU that loads the library holds it until the process exits.
  *     Larger B*H returns SDM_ERR_UNSUPPORTED before any work is enqueued.
  *   - The first call on a device looks up the array's device address (with
- *     that device current); make that first call before any stream capture.
+ *     that device current), and so does the first call in a new CUDA context
+ *     of the device (after cudaDeviceReset, for instance); make that first
+ *     call before any stream capture.
  *   - The call allocates nothing and clears the scratch it uses on `stream`.
  *   - All calls share the one array: calls that overlap on the GPU (another
  *     stream, another thread) race on it and may produce wrong scales.  Order

@@ -85,7 +85,7 @@ def _declare(L):
     L.orc_quantize.argtypes = [_P, _I, _I64, _I, _I, _P, _P]
     L.orc_attention.restype = None
     L.orc_attention.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I64, _I64, _I,
-                                _P, _I64, _I64, _I64, _I, _I, _D, _P, _P, _P]
+                                _P, _I64, _I64, _I64, _I, _I, _D, _D, _P, _P, _P]
     L.orc_attention_exact.restype = None
     L.orc_attention_exact.argtypes = [_P, _P, _P, _I, _I, _I64, _I64, _I, _P, _I64, _P]
     L.orc_num_threads.restype = _I
@@ -180,13 +180,16 @@ ARITH = {"definition": 0, "fp32": 1}
 
 
 def attention(q8, k8, v8, s_q, s_k, s_v, rows=None, bc: int = KV_TILE, split: int = 0,
-              quant_p: bool = True, delta: float = 0.0, arith: str = "definition"):
+              quant_p: bool = True, delta: float = 0.0, kappa: float = 0.0, arith: str = "definition"):
     """FP8 online-softmax attention of the selected rows of q8 to all keys.
 
     q8 [B,H,T,d], k8/v8 [B,H,N,d] uint8 codes; s_* [B,H] fp32.
     arith: "definition" (the oracle: logits, exp and sums in double) or "fp32"
     (a diagnostic: the single-precision sequence a tensor-core kernel takes).
-    Returns (out16 [B,n,H,d] fp16, out [B,n,H,d] f64, ambiguity report [B,n,H,d] f64).
+    delta, kappa: the ambiguity radius delta + kappa * (|m2| + |t_j|) of key j
+    (base-2 units); the returned allowance bounds the output change when any set
+    of keys within that relative distance of an e4m3 midpoint takes its other code.
+    Returns (out16 [B,n,H,d] fp16, out [B,n,H,d] f64, allowance [B,n,H,d] f64).
     """
     q8 = np.ascontiguousarray(q8, np.uint8)
     k8 = np.ascontiguousarray(k8, np.uint8)
@@ -206,7 +209,7 @@ def attention(q8, k8, v8, s_q, s_k, s_v, rows=None, bc: int = KV_TILE, split: in
     allow = np.empty((B, n, H, d), np.float64)
     lib().orc_attention(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(sq), _ptr(sk), _ptr(sv),
                         B, H, T, N, d, _ptr(rows), n, int(bc), int(split),
-                        1 if quant_p else 0, ARITH[arith], float(delta),
+                        1 if quant_p else 0, ARITH[arith], float(delta), float(kappa),
                         _ptr(out16), _ptr(out), _ptr(allow))
     return out16.view(np.float16), out, allow
 
@@ -228,7 +231,8 @@ def attention_exact(q, k, v, rows=None):
     return out
 
 
-def layer(q, k, v, n_ctx: int, c_h, gate=None, rows=None, split: int = 0, delta: float = 0.0):
+def layer(q, k, v, n_ctx: int, c_h, gate=None, rows=None, split: int = 0, delta: float = 0.0,
+          kappa: float = 0.0):
     """All steps of the layer on the CPU: qscale -> scales -> e4m3 -> attention.
 
     q [B,T,H,d] fp16 (T = n_ctx + queries), k/v [B,n_ctx,H,d] fp16.
@@ -241,7 +245,7 @@ def layer(q, k, v, n_ctx: int, c_h, gate=None, rows=None, split: int = 0, delta:
     q8 = quantize(qs, s_q)
     k8 = quantize(k, s_k)
     v8 = quantize(v, s_v)
-    o16, o, allow = attention(q8, k8, v8, s_q, s_k, s_v, rows=rows, split=split, delta=delta)
+    o16, o, allow = attention(q8, k8, v8, s_q, s_k, s_v, rows=rows, split=split, delta=delta, kappa=kappa)
     return dict(q_scaled=qs, s_q=s_q, s_k=s_k, s_v=s_v, q8=q8, k8=k8, v8=v8,
                 out16=o16, out=o, allow=allow)
 
@@ -253,7 +257,7 @@ def _ragged_rows(n_b: int, N: int, T: int) -> np.ndarray:
     return np.concatenate([np.arange(n_b), np.arange(N, T)]).astype(np.int64)
 
 
-def layer_ragged(q, k, v, ctx_len, c_h, gate=None, split: int = 0, delta: float = 0.0):
+def layer_ragged(q, k, v, ctx_len, c_h, gate=None, split: int = 0, delta: float = 0.0, kappa: float = 0.0):
     """A batch of estimators whose contexts are padded to N rows ("unmasked context
     rows", [FP8 3/4] opening section): batch b is `layer` on its own rows only --
     query scaling with n = n_b, scales from rows [0, n_b), context rows [0, n_b)
@@ -277,7 +281,7 @@ def layer_ragged(q, k, v, ctx_len, c_h, gate=None, split: int = 0, delta: float 
         rows = _ragged_rows(n, N, T)
         g = None if gate is None else np.ascontiguousarray(gate[b:b + 1, rows])
         r = layer(np.ascontiguousarray(q[b:b + 1, rows]), np.ascontiguousarray(k[b:b + 1, :n]),
-                  np.ascontiguousarray(v[b:b + 1, :n]), n, c_h, g, split=split, delta=delta)
+                  np.ascontiguousarray(v[b:b + 1, :n]), n, c_h, g, split=split, delta=delta, kappa=kappa)
         for key in ("out16", "out", "allow", "q_scaled"):
             res[key][b, rows] = r[key][0]
         for key in ("s_q", "s_k", "s_v"):

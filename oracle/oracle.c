@@ -272,11 +272,18 @@ static void e4m3_neighbours(uint8_t c, double* lo_mid, double* lo_alt,
  * for the definition), and with quant_p == 0 the e4m3 rounding of P is
  * skipped: the plain softmax.
  *
- * Ambiguity report: keys whose probability lies within relative distance
- * delta of an e4m3 rounding midpoint are ones where an implementation whose
- * probabilities err by that much may pick the other code; amb0 accumulates the
- * weight change that choice would make and amb1[e] that change times
- * |dec(v8_j[e])|, with the same rescaling as l/acc.
+ * Ambiguity allowance.  An implementation that forms the logits in fp32 (a
+ * tensor core accumulates z in fp32; m2 and t are rounded to fp32) moves each
+ * probability by a small relative error, and where the definition's
+ * probability lies that close to an e4m3 rounding midpoint either neighbouring
+ * code is what such an implementation may produce.  For key j the radius is
+ *   r_j = delta0 + kappa * (|m2| + |t_j|)      (base-2 units: m2 the running
+ *                                                maximum, t_j = x_j log2 e - m2)
+ * -- a fixed part for the 2^x evaluation and a part proportional to the size
+ * of the fp32 numbers the logit passes through.  A key whose probability p
+ * lies within relative distance r_j of a midpoint is "ambiguous": amb0
+ * accumulates |dw|, the weight change its other code would make, and amb1[e]
+ * |dw| * |dec(v8_j[e])|, with the same rescaling as l/acc.
  */
 enum { ORC_ARITH_DEFINITION = 0, ORC_ARITH_FP32 = 1 };
 
@@ -295,16 +302,16 @@ static void partial_scale(orc_partial* st, int d, double alpha) {
 /* Adds key j with probability p (>= 0) to the running sums: its e4m3 weight
  * (or p itself when quant_p == 0) and its ambiguity contribution. */
 static void partial_add_key(orc_partial* st, double p, const uint8_t* vj, int d,
-                            int quant_p, double delta) {
+                            int quant_p, double radius) {
     double w = p, dw = 0.0;
     if (quant_p) {
         uint8_t c = orc_e4m3_encode(p);
         w = orc_e4m3_decode(c);
-        if (p > 0.0 && delta > 0.0) {
+        if (p > 0.0 && radius > 0.0) {
             double lo_mid, lo_alt, hi_mid, hi_alt;
             e4m3_neighbours(c, &lo_mid, &lo_alt, &hi_mid, &hi_alt);
-            if (fabs(p - lo_mid) <= delta * p) dw = fabs(w - lo_alt);
-            if (fabs(p - hi_mid) <= delta * p) dw = fabs(hi_alt - w);
+            if (fabs(p - lo_mid) <= radius * p) dw = fabs(w - lo_alt);
+            if (fabs(p - hi_mid) <= radius * p) dw = fabs(hi_alt - w);
         }
     }
     if (w == 0.0 && dw == 0.0) return;
@@ -325,8 +332,8 @@ static const double kLog2e = 1.4426950408889634074;
 
 static void attend_range_definition(const uint8_t* q8row, const uint8_t* k8, const uint8_t* v8,
                                     int64_t j_begin, int64_t j_end, int d, double scale,
-                                    int64_t bc, int quant_p, double delta, orc_partial* st,
-                                    double* xbuf) {
+                                    int64_t bc, int quant_p, double delta0, double kappa,
+                                    orc_partial* st, double* xbuf) {
     double m = -INFINITY;                     /* running max of x (natural-log units) */
     partial_reset(st, d);
     for (int64_t j0 = j_begin; j0 < j_end; j0 += bc) {
@@ -343,16 +350,18 @@ static void attend_range_definition(const uint8_t* q8row, const uint8_t* k8, con
             partial_scale(st, d, m == -INFINITY ? 0.0 : exp(m - mt));
             m = mt;
         }
-        for (int64_t j = j0; j < j1; ++j)
-            partial_add_key(st, exp(xbuf[j - j0] - m), v8 + j * d, d, quant_p, delta);
+        for (int64_t j = j0; j < j1; ++j) {
+            double r = delta0 + kappa * (fabs(m) + (m - xbuf[j - j0])) * kLog2e;
+            partial_add_key(st, exp(xbuf[j - j0] - m), v8 + j * d, d, quant_p, r);
+        }
     }
     st->m2 = m * kLog2e;
 }
 
 static void attend_range_f32(const uint8_t* q8row, const uint8_t* k8, const uint8_t* v8,
                              int64_t j_begin, int64_t j_end, int d, float c2,
-                             int64_t bc, int quant_p, double delta, orc_partial* st,
-                             double* xbuf) {
+                             int64_t bc, int quant_p, double delta0, double kappa,
+                             orc_partial* st, double* xbuf) {
     float m = -INFINITY;                      /* running max of z (raw units) */
     float m2 = -INFINITY;
     partial_reset(st, d);
@@ -373,7 +382,8 @@ static void attend_range_f32(const uint8_t* q8row, const uint8_t* k8, const uint
         }
         for (int64_t j = j0; j < j1; ++j) {
             float t = fmaf((float)xbuf[j - j0], c2, -m2);
-            partial_add_key(st, (double)(float)exp2((double)t), v8 + j * d, d, quant_p, delta);
+            double r = delta0 + kappa * (fabs((double)m2) + fabs((double)t));
+            partial_add_key(st, (double)(float)exp2((double)t), v8 + j * d, d, quant_p, r);
         }
     }
     st->m2 = m2;
@@ -400,17 +410,20 @@ static float softmax_c2(float s_q, float s_k, int d) {
  *   arith              ORC_ARITH_DEFINITION or ORC_ARITH_FP32 (see above)
  *   out16 [B][n_rows][H][d]   fp16 bits of ACC * s_v / L
  *   out   [B][n_rows][H][d]   the same value before fp16 rounding (double)
- *   allow [B][n_rows][H][d]   ambiguity report (may be NULL): first-order
- *                      change of O if every key whose p sits within relative
- *                      delta of an e4m3 midpoint took the other code:
- *                      s_v * (amb1[e] + amb0 * vmax_e) / L, where vmax_e is the
- *                      largest |dec(v8[.][e])| of the head.
+ *   delta0, kappa      radius of the ambiguity allowance (see above); 0, 0: none
+ *   allow [B][n_rows][H][d]   ambiguity allowance (may be NULL): an upper bound
+ *                      on |O' - O| when any subset of the ambiguous keys takes
+ *                      its other code:  s_v * (amb1[e] + amb0 * vmax_e) / (L - amb0)
+ *                      (infinite if amb0 >= L), vmax_e the largest |dec(v8[.][e])|
+ *                      of the head.  Flipping a set S changes the numerator by
+ *                      sum_S dw_j (v_j - O) and L by sum_S dw_j, and
+ *                      |v_j - O| <= |v_j| + vmax_e, L' >= L - amb0.
  */
 void orc_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
                    const float* s_q, const float* s_k, const float* s_v,
                    int B, int H, int64_t T, int64_t N, int d,
                    const int64_t* rows, int64_t n_rows, int64_t bc, int64_t split,
-                   int quant_p, int arith, double delta,
+                   int quant_p, int arith, double delta0, double kappa,
                    uint16_t* out16, double* out, double* allow) {
     int64_t n_chunks = (split > 0) ? (N + split - 1) / split : 1;
     int64_t chunk = (split > 0) ? split : N;
@@ -446,10 +459,11 @@ void orc_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
                 int64_t jb = s * chunk, je = jb + chunk < N ? jb + chunk : N;
                 double ms;
                 if (arith == ORC_ARITH_FP32) {
-                    attend_range_f32(qrow, kb, vb, jb, je, d, c2, bc, quant_p, delta, &st, xbuf);
+                    attend_range_f32(qrow, kb, vb, jb, je, d, c2, bc, quant_p, delta0, kappa, &st, xbuf);
                     ms = st.m2;
                 } else {
-                    attend_range_definition(qrow, kb, vb, jb, je, d, scale, bc, quant_p, delta, &st, xbuf);
+                    attend_range_definition(qrow, kb, vb, jb, je, d, scale, bc, quant_p, delta0, kappa,
+                                            &st, xbuf);
                     ms = st.m2 / kLog2e;      /* back to natural-log units */
                 }
                 if (st.m2 == -INFINITY) continue;
@@ -469,7 +483,9 @@ void orc_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
                 double val = ACC[e] * (double)s_v[bh] / L;
                 if (out) out[o + e] = val;
                 if (out16) out16[o + e] = orc_f16_encode(val);
-                if (allow) allow[o + e] = (double)s_v[bh] * (A1[e] + A0 * vmax[bh * d + e]) / L;
+                if (allow) allow[o + e] = A0 == 0.0 ? 0.0
+                                        : (A0 >= L ? INFINITY
+                                                   : (double)s_v[bh] * (A1[e] + A0 * vmax[bh * d + e]) / (L - A0));
             }
         }
         free(xbuf); free(tmp);

@@ -2,10 +2,11 @@
 
 FP8 tensors and scales are compared bit for bit; attention outputs against the
 oracle's double-precision definition within the specification's gates: every
-element within max(2e-2, one fp16 ulp of its value) and mean |d| <= 1e-3, with
-nothing added for keys whose probability sits next to an e4m3 rounding midpoint
-(the share of such outputs is only reported).  The error against exact
-attention is printed for the record.
+element within max(2e-2, one fp16 ulp of its value) and mean |d| <= 1e-3.  Only
+an output with a key whose probability lies within fp32 rounding distance of an
+e4m3 midpoint (where either code is what a correct single-precision kernel may
+produce) gets the oracle's pinned bound on the change that code choice makes.
+The error against exact attention is printed for the record.
 """
 import os
 
@@ -14,7 +15,7 @@ import pytest
 import torch
 
 from fp8_quant_logscale_b200.workloads import WORKLOADS, make_inputs
-from parity import DELTA, dev, gate, host
+from parity import AMB, dev, gate, host
 
 pytestmark = pytest.mark.gpu
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -61,7 +62,7 @@ def _layer_case(cuda_lib, orc, inp, gated=False, rows=None, report=""):
     assert (host(cache.k8) == k8).all()
     assert (host(cache.v8t)[..., :N] == v8.transpose(0, 1, 3, 2)).all()
     q8 = orc.quantize(qs, s_q)
-    o16, o, allow = orc.attention(q8, k8, v8, s_q, s_k, s_v, rows=rows, delta=DELTA)
+    o16, o, allow = orc.attention(q8, k8, v8, s_q, s_k, s_v, rows=rows, **AMB)
     got = host(out) if rows is None else host(out)[:, rows]
     stats = gate(got, o, allow, report)
     # error against exact attention, reported only: on at most 256 of the checked rows

@@ -5,7 +5,7 @@ import pytest
 import torch
 
 from fp8_quant_logscale_b200.workloads import WORKLOADS, make_inputs
-from parity import DELTA, dev, gate, host
+from parity import AMB, dev, gate, host
 
 pytestmark = pytest.mark.gpu
 
@@ -23,7 +23,7 @@ def _oracle_cached(orc, inp, queries, rows=None):
     s_q, s_k, s_v = (orc.context_scales(x, N) for x in (qs, inp["k"], inp["v"]))
     k8, v8 = orc.quantize(inp["k"], s_k), orc.quantize(inp["v"], s_v)
     qq = orc.quantize(orc.qscale(queries, N, inp["c_h"]), s_q)
-    return orc.attention(qq, k8, v8, s_q, s_k, s_v, rows=rows, split=orc.split_keys(N), delta=DELTA)
+    return orc.attention(qq, k8, v8, s_q, s_k, s_v, rows=rows, split=orc.split_keys(N), **AMB)
 
 
 @pytest.mark.parametrize("N,M,H", [(20000, 300, 3), (16384, 64, 8), (1000, 1, 2), (33000, 129, 4)])
@@ -76,5 +76,5 @@ def test_cached_batch2_gated_queries(cuda_lib, orc):
     s_q, s_k, s_v = (orc.context_scales(x, N) for x in (qs, inp["k"], inp["v"]))
     qq = orc.quantize(orc.qscale(inp["queries"], N, inp["c_h"], g_q), s_q)
     _, o, allow = orc.attention(qq, orc.quantize(inp["k"], s_k), orc.quantize(inp["v"], s_v), s_q, s_k, s_v,
-                                split=orc.split_keys(N), delta=DELTA)
+                                split=orc.split_keys(N), **AMB)
     print("\ncached B2 gated:", gate(out, o, allow, "cached B2 gated"))

@@ -12,7 +12,7 @@ import pytest
 import torch
 
 from fp8_quant_logscale_b200.workloads import WORKLOADS, make_inputs
-from parity import DELTA, dev, gate, host
+from parity import AMB, dev, gate, host
 
 pytestmark = pytest.mark.gpu
 
@@ -77,7 +77,7 @@ def test_offload_ragged_cache(cuda_lib, orc):
         q8 = orc.quantize(orc.qscale(qn[b:b + 1], n, inp["c_h"]), r["s_q"][b:b + 1])
         _, o, allow = orc.attention(q8, np.ascontiguousarray(r["k8"][b:b + 1, :, :n]),
                                     np.ascontiguousarray(r["v8"][b:b + 1, :, :n]), r["s_q"][b:b + 1],
-                                    r["s_k"][b:b + 1], r["s_v"][b:b + 1], split=orc.split_keys(N), delta=DELTA)
+                                    r["s_k"][b:b + 1], r["s_v"][b:b + 1], split=orc.split_keys(N), **AMB)
         print(f"\noffload ragged batch {b} n_b={n}:", gate(got[b:b + 1], o, allow, f"offload ragged b{b}"))
 
 
@@ -103,7 +103,7 @@ def test_offload_full_size(cuda_lib, orc):
     s_q, s_k, s_v = (orc.context_scales(x, N) for x in (qs, inp["k"], inp["v"]))
     q8 = orc.quantize(orc.qscale(inp["queries"], N, inp["c_h"]), s_q)
     _, o, allow = orc.attention(q8, orc.quantize(inp["k"], s_k), orc.quantize(inp["v"], s_v), s_q, s_k, s_v,
-                                rows=rows, split=orc.split_keys(N), delta=DELTA)
+                                rows=rows, split=orc.split_keys(N), **AMB)
     print("\noffload 512K, 256 queries:", gate(host(got)[:, rows], o, allow, "offload 512K"))
 
 

@@ -66,7 +66,7 @@ def test_query_rows_above_the_context_amax_saturate(cuda_lib, orc):
     context value quantise to the saturated codes +-448 (0x7E / 0xFE); the codes
     match the oracle bit for bit and the layer's outputs for those rows stay
     within the gates."""
-    from parity import DELTA, gate
+    from parity import AMB, gate
     N, M, H = 1000, 100, 3
     inp = make_inputs(WORKLOADS["icl_n1k_m128_h4"], n_ctx=N, n_query=M, heads=H)
     q = inp["q"].astype(np.float32)
@@ -81,5 +81,5 @@ def test_query_rows_above_the_context_amax_saturate(cuda_lib, orc):
     torch.cuda.synchronize()
     assert (host(q8) == want).all()
     out = cuda_lib.icl_attention(dev(q), dev(inp["k"]), dev(inp["v"]), N, dev(inp["c_h"]))
-    ref = orc.layer(q, inp["k"], inp["v"], N, inp["c_h"], delta=DELTA)
+    ref = orc.layer(q, inp["k"], inp["v"], N, inp["c_h"], **AMB)
     gate(host(out), ref["out"], ref["allow"], "saturated query rows")

@@ -8,7 +8,7 @@ import pytest
 import torch
 
 from fp8_quant_logscale_b200.workloads import WORKLOADS, make_inputs
-from parity import DELTA, dev, gate, host
+from parity import AMB, dev, gate, host
 from test_gpu_attention_f16 import check_f16, f16_bound
 
 pytestmark = pytest.mark.gpu
@@ -45,7 +45,7 @@ def test_ragged_fit_parity(cuda_lib, orc, B, N, M, H, lens):
         inp["ctx_len"] = np.array(lens, np.int64)
     inp = poison_padding(inp)
     out, cache = fit_ragged(cuda_lib, inp)
-    r = orc.layer_ragged(inp["q"], inp["k"], inp["v"], inp["ctx_len"], inp["c_h"], delta=DELTA)
+    r = orc.layer_ragged(inp["q"], inp["k"], inp["v"], inp["ctx_len"], inp["c_h"], **AMB)
     sc = host(cache.scales)
     assert (sc[0] == r["s_q"]).all() and (sc[1] == r["s_k"]).all() and (sc[2] == r["s_v"]).all()
     assert (host(cache.k8) == r["k8"]).all()
@@ -63,7 +63,7 @@ def test_ragged_gated(cuda_lib, orc):
     inp["gate"] = make_inputs(WORKLOADS["icl_n128k_m1k_h8_gated"], n_ctx=700, n_query=40, heads=2,
                               batch=3)["gate"]
     out, cache = fit_ragged(cuda_lib, inp, gated=True)
-    r = orc.layer_ragged(inp["q"], inp["k"], inp["v"], inp["ctx_len"], inp["c_h"], inp["gate"], delta=DELTA)
+    r = orc.layer_ragged(inp["q"], inp["k"], inp["v"], inp["ctx_len"], inp["c_h"], inp["gate"], **AMB)
     assert (host(cache.scales)[0] == r["s_q"]).all()
     gate(out, r["out"], r["allow"], "ragged gated")
 
@@ -95,7 +95,7 @@ def test_cached_prediction_against_a_ragged_cache(cuda_lib, orc):
         k8 = np.ascontiguousarray(r["k8"][b:b + 1, :, :n])
         v8 = np.ascontiguousarray(r["v8"][b:b + 1, :, :n])
         o16, o, allow = orc.attention(q8, k8, v8, r["s_q"][b:b + 1], r["s_k"][b:b + 1], r["s_v"][b:b + 1],
-                                      split=L, delta=DELTA)
+                                      split=L, **AMB)
         gate(pred[b:b + 1], o, allow, f"cached ragged batch {b} n_b={n}")
     # batch invariance: one query at a time gives the same bits
     one = host(cuda_lib.cached_attention(dev(queries[:, 5:6].copy()), cache, dev(inp["c_h"])))
@@ -133,7 +133,7 @@ def test_full_size_ragged_workload_sampled(cuda_lib, orc):
         rows_b = np.r_[0:n, N:N + M]
         sel = np.unique(np.r_[np.arange(0, rows_b.size, 97), [n - 1, n, rows_b.size - 1]]).astype(np.int64)
         r = orc.layer(np.ascontiguousarray(inp["q"][b:b + 1, rows_b]), np.ascontiguousarray(inp["k"][b:b + 1, :n]),
-                      np.ascontiguousarray(inp["v"][b:b + 1, :n]), n, inp["c_h"], rows=sel, delta=DELTA)
+                      np.ascontiguousarray(inp["v"][b:b + 1, :n]), n, inp["c_h"], rows=sel, **AMB)
         assert (sc[0][b] == r["s_q"][0]).all() and (sc[1][b] == r["s_k"][0]).all()
         gate(out[b:b + 1, rows_b[sel]], r["out"], r["allow"], f"full ragged batch {b} n_b={n}")
 

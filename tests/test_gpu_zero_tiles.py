@@ -14,7 +14,7 @@ input.
 import numpy as np
 import pytest
 
-from parity import DELTA, dev, gate, host
+from parity import AMB, dev, gate, host
 
 pytestmark = pytest.mark.gpu
 LOG2E = 1.4426950408889634
@@ -79,7 +79,7 @@ def test_zero_tiles_one_call(cuda_lib, orc):
                                  ws=ws)
     st, flags = cuda_lib.sync_status(ws)
     assert st == 0 and flags == 0, (st, flags)
-    ref = orc.layer(inp["q"], inp["k"], inp["v"], N, inp["c_h"], delta=DELTA)
+    ref = orc.layer(inp["q"], inp["k"], inp["v"], N, inp["c_h"], **AMB)
     stats = gate(host(out), ref["out"], ref["allow"], "zero tiles, one call")
     print(f"\nzero tiles one call: {stats}")
 
@@ -102,6 +102,6 @@ def test_zero_tiles_split_kv(cuda_lib, orc, n_pred):
     s_q, s_k, s_v = (orc.context_scales(x, N) for x in (qs, inp["k"], inp["v"]))
     k8, v8 = orc.quantize(inp["k"], s_k), orc.quantize(inp["v"], s_v)
     qq = orc.quantize(orc.qscale(queries, N, inp["c_h"]), s_q)
-    _, o, allow = orc.attention(qq, k8, v8, s_q, s_k, s_v, split=split, delta=DELTA)
+    _, o, allow = orc.attention(qq, k8, v8, s_q, s_k, s_v, split=split, **AMB)
     stats = gate(pred, o, allow, f"zero tiles, split-KV, {n_pred} queries")
     print(f"\nzero tiles split-KV, {n_pred} queries: {stats}")

@@ -243,7 +243,97 @@ def test_allowance_properties(orc):
     _, _, a0 = orc.attention(q8, k8, v8, sq, sk, sv, delta=0.0)
     _, _, a1 = orc.attention(q8, k8, v8, sq, sk, sv, delta=1e-4)
     _, _, a2 = orc.attention(q8, k8, v8, sq, sk, sv, delta=1e-2)
-    assert (a0 == 0).all() and (a1 >= 0).all() and (a2 >= a1).all() and a2.max() > 0
+    _, _, a3 = orc.attention(q8, k8, v8, sq, sk, sv, delta=1e-4, kappa=1e-4)
+    assert (a0 == 0).all() and (a1 >= 0).all() and (a2 >= a1).all() and a2.max() > 0 and (a3 >= a1).all()
+
+
+_E4M3_POS = np.unique(_torch_e4m3_decode(np.arange(0x7F, dtype=np.uint8)))    # 0 .. 448, every value
+
+
+def _flips(orc, q8, k8, v8, sq, sk, sv, bc, split, delta, kappa, n_random, seed):
+    """Brute force on the materialised definition: for every (row, head), the keys whose
+    probability lies within relative r_j = delta + kappa (|m2| + |t_j|) of an e4m3 midpoint
+    (found here from the value grid, independently of the oracle); flip each alone, all of
+    them together and random subsets to the other neighbouring code, and return the
+    largest |O' - O| / allowance over all of them (must be <= 1)."""
+    q, k, v = (_torch_e4m3_decode(c) for c in (q8, k8, v8))
+    B, H, T, _ = q.shape
+    N = k.shape[2]
+    x = (q @ k.transpose(0, 1, 3, 2)) * (sq.astype(np.float64) * sk.astype(np.float64) / 8.0)[..., None, None]
+    chunk = split if split > 0 else N
+    run = np.empty_like(x)
+    for c0 in range(0, N, chunk):
+        m = np.full(x.shape[:-1], -np.inf)
+        for j0 in range(c0, min(N, c0 + chunk), bc):
+            j1 = min(j0 + bc, c0 + chunk, N)
+            m = np.maximum(m, x[..., j0:j1].max(-1))
+            run[..., j0:j1] = m[..., None]
+    M = x.max(-1, keepdims=True)
+    p = np.exp(x - run)
+    val = _e4m3_round(p)
+    idx = np.searchsorted(_E4M3_POS, val)
+    below = _E4M3_POS[np.maximum(idx - 1, 0)]
+    above = _E4M3_POS[np.minimum(idx + 1, _E4M3_POS.size - 1)]
+    r = delta + kappa * (np.abs(run) + (run - x)) * LOG2E
+    lo = (np.abs(p - (val + below) / 2) <= r * p) & (val > 0)
+    hi = np.abs(p - (val + above) / 2) <= r * p
+    alt = np.where(hi, above, np.where(lo, below, val))
+    amb = lo | hi
+    _, _, allow = orc.attention(q8, k8, v8, sq, sk, sv, bc=bc, split=split, delta=delta, kappa=kappa)
+    allow = allow.transpose(0, 2, 1, 3)                                    # [B,H,T,d]
+    scale = np.exp(run - M)
+    o = ((val * scale) @ v) / (val * scale).sum(-1, keepdims=True)
+    rng = np.random.default_rng(seed)
+    worst, n_amb = 0.0, int(amb.sum())
+    for b in range(B):
+        for h in range(H):
+            for i in range(T):
+                keys = np.nonzero(amb[b, h, i])[0]
+                if keys.size == 0:
+                    continue
+                sets = [[j] for j in keys] + [list(keys)]
+                sets += [list(rng.choice(keys, rng.integers(1, keys.size + 1), replace=False))
+                         for _ in range(n_random)]
+                for S in sets:
+                    w = val[b, h, i].copy()
+                    w[S] = alt[b, h, i, S]
+                    w *= scale[b, h, i]
+                    o2 = (w @ v[b, h]) / w.sum()
+                    d = np.abs(o2 - o[b, h, i]) * float(sv[b, h])
+                    worst = max(worst, float((d / np.maximum(allow[b, h, i], 1e-300)).max()))
+    return worst, n_amb
+
+
+@pytest.mark.parametrize("bc,split,delta,kappa", [(200, 0, 2e-2, 0.0), (7, 0, 1e-2, 0.0), (32, 96, 3e-3, 1e-3),
+                                                  (128, 0, 1e-3, 3e-3)])
+def test_allowance_bounds_every_flip(orc, bc, split, delta, kappa):
+    """The allowance is an upper bound on the output change of any set of ambiguous keys
+    taking their other code (a large radius makes many keys ambiguous)."""
+    q8, k8, v8, sq, sk, sv = _problem(orc, T=24, N=200, seed=31, qscale=1.0)
+    worst, n_amb = _flips(orc, q8, k8, v8, sq, sk, sv, bc, split, delta, kappa, n_random=8, seed=1)
+    assert n_amb > 100, n_amb
+    assert worst <= 1.0, worst
+
+
+def test_allowance_bounds_flips_of_keys_far_from_the_output(orc):
+    """V rows around 3 with a third of them zero: flipping a key whose value is 0 moves O
+    by its whole size, which the allowance's vmax term covers."""
+    q8, k8, _, sq, sk, _ = _problem(orc, T=24, N=200, seed=37, qscale=3.0)
+    rng = np.random.default_rng(41)
+    v = (3.0 + 0.5 * rng.standard_normal((1, 200, 2, 64))).astype(np.float16)
+    v[:, rng.random(200) < 0.33] = 0
+    sv = orc.context_scales(v, 200)
+    v8 = orc.quantize(v, sv)
+    worst, n_amb = _flips(orc, q8, k8, v8, sq, sk, sv, 128, 0, 2e-2, 0.0, n_random=8, seed=2)
+    assert n_amb > 100 and worst <= 1.0, (n_amb, worst)
+
+
+def test_allowance_is_not_vacuous(orc):
+    """The bound is within a factor 10 of a change some flip actually makes, so an
+    allowance ten times too small would fail the brute force above."""
+    q8, k8, v8, sq, sk, sv = _problem(orc, T=24, N=200, seed=31, qscale=1.0)
+    worst, _ = _flips(orc, q8, k8, v8, sq, sk, sv, 200, 0, 2e-2, 0.0, n_random=0, seed=1)
+    assert worst > 0.1, worst
 
 
 def test_lossless_when_inputs_are_e4m3_values(orc):
