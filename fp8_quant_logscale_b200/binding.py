@@ -30,7 +30,7 @@ EXPORTS = ("sdm_status_string", "sdm_version", "sdm_split_keys", "sdm_cache_layo
            "sdm_cached_attention", "sdm_fp8_eligible", "sdm_icl_attention_f16", "sdm_icl_attention_ragged",
            "sdm_icl_attention_f16_ragged", "sdm_cached_attention_offload", "sdm_gqa_prefill",
            "sdm_gqa_prefill_workspace_size", "sdm_sync_status",
-           "sdm_selftest_wait_timeout")
+           "sdm_selftest_wait_timeout", "sdm_context_amax", "sdm_quantize_with_scales", "sdm_cache_put_rows")
 NOALLOC_MAX_BATCH_HEADS = 4096
 
 
@@ -107,6 +107,13 @@ def lib() -> ctypes.CDLL:
         L.sdm_selftest_wait_timeout.argtypes = [_P, _I64, _P]
         L.sdm_sync_status.restype = ctypes.c_int
         L.sdm_sync_status.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_uint32)]
+        L.sdm_context_amax.restype = ctypes.c_int
+        L.sdm_context_amax.argtypes = [_P, _P, _P, _I32, _I64, _I64, _I32, _I32, _I64, _P, _P, _P, _P]
+        L.sdm_quantize_with_scales.restype = ctypes.c_int
+        L.sdm_quantize_with_scales.argtypes = [_P, _P, _P, _I32, _I64, _I64, _I32, _I32, _I64, _P, _P, _P, _P,
+                                               _P, _P, _I64, _P, _I64, _P]
+        L.sdm_cache_put_rows.restype = ctypes.c_int
+        L.sdm_cache_put_rows.argtypes = [ctypes.POINTER(CacheStruct), _P, _I64, _P, _I64, _I64, _I64, _P]
         _lib = L
     return _lib
 
@@ -480,3 +487,69 @@ def gqa_prefill_workspace_size(qo_indptr, kv_indptr, q_heads: int, kv_heads: int
     kvo = (ctypes.c_int64 * len(kv_indptr))(*[int(x) for x in kv_indptr])
     return int(lib().sdm_gqa_prefill_workspace_size(qo, kvo, len(qo_indptr) - 1, q_heads, kv_heads, 128,
                                                     1 if causal else 0))
+
+
+# ------------------------------------------------------ sharded quantisation
+
+def context_amax(q: torch.Tensor, k: torch.Tensor | None, v: torch.Tensor | None, n_ctx: int, n_len: int,
+                 c_h: torch.Tensor | None = None, gate: torch.Tensor | None = None,
+                 out: torch.Tensor | None = None) -> torch.Tensor:
+    """[3, B, H] fp32 maxima of |Q'|, |K|, |V| over context rows [0, n_ctx) of a slice
+    (sdm_context_amax).  q [B, q_rows, H, 64] is raw (query scaling with n_len, c_h,
+    gate fused) or, with c_h None, already scaled."""
+    _want(q, torch.float16, "q", 4)
+    B, q_rows, H, d = q.shape
+    if n_ctx > 0:
+        _want(k, torch.float16, "k", 4)
+        _want(v, torch.float16, "v", 4)
+    if c_h is not None:
+        _want(c_h, torch.float32, "c_h", 1)
+    if gate is not None:
+        _want(gate, torch.float16, "gate", 3)
+    dev = q.device
+    out = torch.empty((3, B, H), dtype=torch.float32, device=dev) if out is None else out
+    with torch.cuda.device(dev):
+        _check(lib().sdm_context_amax(_ptr(q), _ptr(k if n_ctx > 0 else None), _ptr(v if n_ctx > 0 else None), B,
+                                      int(n_ctx), q_rows, H, d, int(n_len), _ptr(c_h), _ptr(gate), _ptr(out),
+                                      _stream(dev)), "sdm_context_amax")
+    return out
+
+
+def quantize_with_scales(q: torch.Tensor, k: torch.Tensor | None, v: torch.Tensor | None, n_ctx: int, n_len: int,
+                         amax: torch.Tensor, c_h: torch.Tensor | None = None, gate: torch.Tensor | None = None,
+                         ld_k: int | None = None, ld_v: int | None = None, scales: torch.Tensor | None = None):
+    """Scales amax/448 and the e4m3 codes of a slice's rows (sdm_quantize_with_scales).
+    q [B, n_ctx + n_query, H, 64]; k, v [B, n_ctx, H, 64].  Returns (q8 [B,H,T,64],
+    k8 [B,H,ld_k,64] (rows [0, n_ctx) written), v8t [B,H,64,ld_v], scales [3,B,H])."""
+    _want(q, torch.float16, "q", 4)
+    _want(amax, torch.float32, "amax", 3)
+    B, T, H, d = q.shape
+    dev = q.device
+    ld_k = n_ctx if ld_k is None else int(ld_k)
+    ld_v = max(KV_TILE, -(-n_ctx // KV_TILE) * KV_TILE) if ld_v is None else int(ld_v)
+    q8 = torch.empty((B, H, T, d), dtype=torch.uint8, device=dev)
+    k8 = torch.empty((B, H, ld_k, d), dtype=torch.uint8, device=dev)
+    v8t = torch.empty((B, H, d, ld_v), dtype=torch.uint8, device=dev)
+    scales = torch.empty((3, B, H), dtype=torch.float32, device=dev) if scales is None else scales
+    if n_ctx > 0:
+        _want(k, torch.float16, "k", 4)
+        _want(v, torch.float16, "v", 4)
+    with torch.cuda.device(dev):
+        _check(lib().sdm_quantize_with_scales(_ptr(q), _ptr(k if n_ctx > 0 else None), _ptr(v if n_ctx > 0 else None),
+                                              B, int(n_ctx), T - int(n_ctx), H, d, int(n_len), _ptr(c_h), _ptr(gate),
+                                              _ptr(amax), _ptr(scales), _ptr(q8),
+                                              _ptr(k8 if n_ctx > 0 else None), ld_k,
+                                              _ptr(v8t if n_ctx > 0 else None), ld_v, _stream(dev)),
+               "sdm_quantize_with_scales")
+    return q8, k8, v8t, scales
+
+
+def cache_put_rows(cache: FP8Cache, k8_rows: torch.Tensor, v8t_cols: torch.Tensor, row0: int, n: int) -> None:
+    """Place rows [0, n) of a slice's K8 planes [B,H,ld_k,64] and columns [0, n) of its
+    V8^T rows [B,H,64,ld_v] at global context row row0 of the cache (sdm_cache_put_rows)."""
+    _want(k8_rows, torch.uint8, "k8_rows", 4)
+    _want(v8t_cols, torch.uint8, "v8t_cols", 4)
+    dev = k8_rows.device
+    with torch.cuda.device(dev):
+        _check(lib().sdm_cache_put_rows(ctypes.byref(cache.struct), _ptr(k8_rows), k8_rows.shape[2], _ptr(v8t_cols),
+                                        v8t_cols.shape[3], int(row0), int(n), _stream(dev)), "sdm_cache_put_rows")

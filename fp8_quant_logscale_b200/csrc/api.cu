@@ -770,6 +770,109 @@ sdm_status sdm_gqa_prefill(const void* q, const void* k, const void* v, const in
   return SDM_OK;
 }
 
+// ---------------------------------------------------------------- sharded step 2
+// Argument checks shared by sdm_context_amax and sdm_quantize_with_scales: the
+// query-scaling inputs (c_h == NULL: q is already scaled) and the slice tensors.
+static sdm_status check_slice(const void* q, const void* k, const void* v, int64_t n_ctx, int64_t n_len,
+                              const float* c_h, const void* gate, int dev) {
+  SDM_TRY(check_tensor(q, dev));
+  if (n_ctx > 0) {
+    SDM_TRY(check_tensor(k, dev));
+    SDM_TRY(check_tensor(v, dev));
+  }
+  if (c_h != nullptr) {
+    if (n_len < 1 || !aligned(c_h, 4)) return SDM_ERR_INVALID_ARG;
+    if (!on_device(c_h, dev)) return SDM_ERR_DEVICE_MISMATCH;
+    if (gate != nullptr) {
+      if (!aligned(gate, 2)) return SDM_ERR_INVALID_ARG;
+      if (!on_device(gate, dev)) return SDM_ERR_DEVICE_MISMATCH;
+    }
+  }
+  return SDM_OK;
+}
+
+static QScale slice_qscale(int64_t n_len, const float* c_h, const void* gate) {
+  // the gate factors are evaluated in place (no workspace to hold them)
+  return c_h != nullptr ? make_qscale(n_len, c_h, gate) : no_qscale();
+}
+
+sdm_status sdm_context_amax(const void* q, const void* k, const void* v, int32_t B, int64_t n_ctx, int64_t q_rows,
+                            int32_t H, int32_t d, int64_t n_len, const float* c_h, const void* gate, float* amax,
+                            void* stream) {
+  SDM_TRY(check_shape(B, n_ctx, q_rows, H, d));
+  if (q_rows < n_ctx) return SDM_ERR_INVALID_ARG;
+  const int dev = current_device();
+  if (dev < 0) return SDM_ERR_CUDA;
+  if (n_ctx > 0) SDM_TRY(check_slice(q, k, v, n_ctx, n_len, c_h, gate, dev));
+  SDM_TRY(check_tensor(amax, dev));
+  cudaStream_t st = as_stream(stream);
+  uint32_t* words = reinterpret_cast<uint32_t*>(amax);  // fp32 bits of values >= 0: integer max = float max
+  SDM_CUDA(cudaMemsetAsync(words, 0, 3 * (size_t)B * H * sizeof(uint32_t), st));
+  if (n_ctx == 0) return SDM_OK;
+  RowsDesc dq{reinterpret_cast<const __half*>(q), B, H, q_rows};
+  RowsDesc dk{reinterpret_cast<const __half*>(k), B, H, n_ctx};
+  RowsDesc dv{reinterpret_cast<const __half*>(v), B, H, n_ctx};
+  SDM_CUDA(launch_context_amax(dq, slice_qscale(n_len, c_h, gate), dk, dv, n_ctx, nullptr, words, st));
+  return SDM_OK;
+}
+
+sdm_status sdm_quantize_with_scales(const void* q, const void* k, const void* v, int32_t B, int64_t n_ctx,
+                                    int64_t n_query, int32_t H, int32_t d, int64_t n_len, const float* c_h,
+                                    const void* gate, const float* amax, float* scales, uint8_t* q8, uint8_t* k8,
+                                    int64_t ld_k, uint8_t* v8t, int64_t ld_v, void* stream) {
+  SDM_TRY(check_shape(B, n_ctx, n_query, H, d));
+  const int64_t T = n_ctx + n_query;
+  if (n_ctx > 0 && (ld_k < n_ctx || ld_k > ((int64_t)1 << 30) || ld_v < n_ctx || ld_v % kKvTile != 0))
+    return SDM_ERR_INVALID_ARG;
+  const int dev = current_device();
+  if (dev < 0) return SDM_ERR_CUDA;
+  if (T > 0) {
+    SDM_TRY(check_slice(q, k, v, n_ctx, n_len, c_h, gate, dev));
+    SDM_TRY(check_tensor(q8, dev));
+  }
+  SDM_TRY(check_tensor(amax, dev));
+  SDM_TRY(check_tensor(scales, dev));
+  if (n_ctx > 0) {
+    SDM_TRY(check_tensor(k8, dev));
+    SDM_TRY(check_tensor(v8t, dev));
+  }
+  cudaStream_t st = as_stream(stream);
+  const int64_t BH = (int64_t)B * H;
+  SDM_CUDA(launch_scales_from_amax(reinterpret_cast<const uint32_t*>(amax), B * H, scales, st));
+  if (T == 0) return SDM_OK;
+  RowsDesc dq{reinterpret_cast<const __half*>(q), B, H, T};
+  SDM_CUDA(launch_quantize_rows(dq, slice_qscale(n_len, c_h, gate), T, scales, q8, T, nullptr, 0, st));
+  if (n_ctx > 0) {
+    RowsDesc dk{reinterpret_cast<const __half*>(k), B, H, n_ctx};
+    RowsDesc dv{reinterpret_cast<const __half*>(v), B, H, n_ctx};
+    SDM_CUDA(launch_quantize_rows(dk, no_qscale(), n_ctx, scales + BH, k8, ld_k, nullptr, 0, st));
+    SDM_CUDA(launch_quantize_vt(dv, n_ctx, nullptr, scales + 2 * BH, v8t, ld_v, st));
+  }
+  return SDM_OK;
+}
+
+sdm_status sdm_cache_put_rows(sdm_fp8_cache* cache, const uint8_t* k8_rows, int64_t ld_k, const uint8_t* v8t_cols,
+                              int64_t ld_v, int64_t row0, int64_t n, void* stream) {
+  if (cache == nullptr) return SDM_ERR_INVALID_ARG;
+  const int dev = current_device();
+  if (dev < 0) return SDM_ERR_CUDA;
+  SDM_TRY(check_cache(cache, cache->batch, cache->heads, cache->head_dim, dev, false));
+  if (n < 0 || row0 < 0 || row0 + n > cache->n_ctx || ld_k < n || ld_v < n) return SDM_ERR_INVALID_ARG;
+  if (n == 0) return SDM_OK;
+  SDM_TRY(check_tensor(k8_rows, dev));
+  SDM_TRY(check_tensor(v8t_cols, dev));
+  cudaStream_t st = as_stream(stream);
+  const int64_t BH = (int64_t)cache->batch * cache->heads;
+  const int64_t N = cache->n_ctx;
+  // K8: one block of n rows (n*64 bytes) per (b, h) plane
+  SDM_CUDA(cudaMemcpy2DAsync(cache->k8 + row0 * kHeadDim, (size_t)N * kHeadDim, k8_rows, (size_t)ld_k * kHeadDim,
+                             (size_t)n * kHeadDim, (size_t)BH, cudaMemcpyDeviceToDevice, st));
+  // V8^T: n columns of each of the B*H*64 rows
+  SDM_CUDA(cudaMemcpy2DAsync(cache->v8t + row0, (size_t)cache->ld_v, v8t_cols, (size_t)ld_v, (size_t)n,
+                             (size_t)BH * kHeadDim, cudaMemcpyDeviceToDevice, st));
+  return SDM_OK;
+}
+
 sdm_status sdm_selftest_wait_timeout(void* ws, int64_t limit_cycles, void* stream) {
   if (ws == nullptr || !aligned(ws, 256)) return SDM_ERR_INVALID_ARG;
   if (limit_cycles < 1000 || limit_cycles > ((int64_t)1 << 31)) return SDM_ERR_INVALID_ARG;

@@ -348,6 +348,82 @@ sdm_status sdm_fp8_quantize_context_noalloc(const void* q_scaled, const void* k,
                                             uint8_t* q8, sdm_fp8_cache* cache, void* stream);
 
 /*
+ * Step 2 split over ranks (one process per GPU), each holding a slice of the
+ * context rows.  The scales are derived from ALL context rows ("[FP8 3/4]
+ * Integrate FP8 attention and caching into TabICLv2", opening section:
+ * context-derived per-head scales); the maximum is exact and associative, so
+ * per-slice maxima combined by an all-reduce(MAX) give the one-process scales
+ * bit for bit.  The pages describe no multi-GPU scheme; this split is the
+ * library's.  A sharded layer call is:
+ *   1. sdm_context_amax on each rank's context slice;
+ *   2. all-reduce(MAX) of the [3][B][H] fp32 words over the ranks (NCCL);
+ *   3. sdm_quantize_with_scales of each rank's rows with the reduced words;
+ *   4. all-gather of the K8 rows and V8^T columns; sdm_cache_put_rows places
+ *      each rank's slice into a full cache on every rank;
+ *   5. sdm_fp8_attention of each rank's quantised rows against that cache.
+ * Each row's result equals the one-process layer's bit for bit.
+ */
+
+/*
+ * Per-(tensor, batch, head) maxima of |Q'|, |K|, |V| over context rows
+ * [0, n_ctx) of this slice.
+ *   q      [B][q_rows][H][d] fp16, q_rows >= n_ctx: raw q (query scaling with the
+ *          global context length n_len, coefficients c_h and optional gate
+ *          [B][q_rows][H] fused, as in sdm_icl_attention) or, with c_h == NULL,
+ *          already-scaled q' (n_len and gate are then ignored)
+ *   k, v   [B][n_ctx][H][d] fp16 (may be NULL when n_ctx == 0)
+ *   amax   out, [3][B][H] fp32 device (values >= 0: Q', K, V); overwritten.
+ *          n_ctx == 0 gives zeros (the identity of the MAX reduction).
+ * No workspace.  Errors: SDM_ERR_INVALID_ARG (null/misaligned pointer,
+ * q_rows < n_ctx, n_len < 1 with c_h), SDM_ERR_UNSUPPORTED (d != 64, heads
+ * outside 1..128), SDM_ERR_DEVICE_MISMATCH; all before any work is enqueued.
+ */
+sdm_status sdm_context_amax(const void* q, const void* k, const void* v, int32_t batch, int64_t n_ctx,
+                            int64_t q_rows, int32_t heads, int32_t head_dim, int64_t n_len, const float* c_h,
+                            const void* gate, float* amax, void* stream);
+
+/*
+ * Scales from the (reduced) maxima and e4m3 codes of this slice's rows:
+ *   scales[t][b][h] = amax[t][b][h] / 448 (IEEE fp32 division; 1 where the
+ *   maximum is 0), the same words sdm_fp8_quantize_context writes;
+ *   q8  [B][H][n_ctx + n_query][d]  e4m3 of the slice's rows of Q' (context rows
+ *       first, then its query rows; query rows above the context maximum
+ *       saturate to +-448)
+ *   k8  [B][H][ld_k][d]             e4m3 of K in rows [0, n_ctx) of each (b, h)
+ *                                   plane, ld_k >= n_ctx (rows past n_ctx are not
+ *                                   written); may be NULL when n_ctx == 0
+ *   v8t [B][H][d][ld_v]             e4m3 of V transposed; ld_v a multiple of 128,
+ *                                   >= n_ctx; columns [n_ctx, ld_v) written zero
+ *   q, k, v, n_len, c_h, gate as for sdm_context_amax, with q holding
+ *   n_ctx + n_query rows.  amax and scales are fp32 [3][B][H] device arrays.
+ * No workspace.  Errors as sdm_context_amax, plus SDM_ERR_INVALID_ARG for a bad
+ * ld_k or ld_v.
+ */
+sdm_status sdm_quantize_with_scales(const void* q, const void* k, const void* v, int32_t batch, int64_t n_ctx,
+                                    int64_t n_query, int32_t heads, int32_t head_dim, int64_t n_len,
+                                    const float* c_h, const void* gate, const float* amax, float* scales,
+                                    uint8_t* q8, uint8_t* k8, int64_t ld_k, uint8_t* v8t, int64_t ld_v,
+                                    void* stream);
+
+/*
+ * Copies a slice of n context rows into a cache at global row `row0`:
+ *   k8_rows  [B][H][ld_k][d] e4m3, rows [0, n) of each plane
+ *            -> cache->k8 rows [row0, row0 + n) of every (b, h)
+ *   v8t_cols [B][H][d][ld_v] e4m3, columns [0, n) of each row
+ *            -> cache->v8t columns [row0, row0 + n)
+ * (device memory of the cache's device; ld_k, ld_v >= n).  The cache's scales
+ * block is not touched, and `filled` is not set: the caller writes the scales
+ * (sdm_quantize_with_scales) and sets filled = 1 once every slice is in.
+ * Columns [N, ld_v) of cache->v8t must be zero (the caller zero-fills the
+ * buffer once).  Two strided device-to-device copies on `stream`.
+ * Errors: SDM_ERR_INVALID_ARG (row range outside [0, N), ld_k or ld_v < n,
+ * null or misaligned pointers), SDM_ERR_CACHE_MISMATCH (cache on another
+ * device), SDM_ERR_CUDA.
+ */
+sdm_status sdm_cache_put_rows(sdm_fp8_cache* cache, const uint8_t* k8_rows, int64_t ld_k, const uint8_t* v8t_cols,
+                              int64_t ld_v, int64_t row0, int64_t n, void* stream);
+
+/*
  * Wait for `stream`, then read and clear the device error word at the head of
  * a workspace used by the calls above.  Returns SDM_OK, SDM_ERR_TIMEOUT (an
  * in-kernel wait gave up; `*flags` gets the raw bits if flags != NULL) or

@@ -50,3 +50,83 @@ def test_max_over_ranks_and_rank0_output():
     res = [json.loads(o.strip().splitlines()[-1]) for o, _ in outs]
     assert all(r["max"] == 2.5 for r in res)
     assert res[1]["ref_out"] == ""   # non-zero ranks print nothing in the reference arm
+
+
+SHARD_CHILD = r'''
+import os, sys, json
+sys.path.insert(0, sys.argv[1])
+import numpy as np
+import torch
+import torch.distributed as dist
+import oracle as orc
+from fp8_quant_logscale_b200.sharded import shard_range
+from fp8_quant_logscale_b200.workloads import WORKLOADS, make_inputs
+
+dist.init_process_group("gloo")
+G, r = dist.get_world_size(), dist.get_rank()
+N, M, H, B = 700, 45, 3, 2
+inp = make_inputs(WORKLOADS["icl_n128k_m1k_h8_gated"], n_ctx=N, n_query=M, heads=H, batch=B)
+c0, c1 = shard_range(N, G, r)
+q0, q1 = shard_range(M, G, r)
+rows = np.r_[c0:c1, N + q0:N + q1]
+n_r = c1 - c0
+# this rank's data only: its context rows and query rows of q (and gate), its rows of k, v
+q_loc, g_loc = inp["q"][:, rows], inp["gate"][:, rows]
+k_loc, v_loc = inp["k"][:, c0:c1], inp["v"][:, c0:c1]
+# 1. query scaling with the global length, maxima over the local context rows
+qs_loc = orc.qscale(np.ascontiguousarray(q_loc), N, inp["c_h"], np.ascontiguousarray(g_loc))
+amax = torch.from_numpy(np.stack([np.abs(x[:, :n_r].astype(np.float32)).max(axis=(1, 3))
+                                  for x in (qs_loc, k_loc, v_loc)]))
+# 2. all-reduce(MAX)
+dist.all_reduce(amax, op=dist.ReduceOp.MAX)
+scales = (amax.numpy() / np.float32(448.0)).astype(np.float32)
+scales[amax.numpy() == 0] = 1.0
+# 3. codes of the local rows with the reduced scales
+q8_loc = orc.quantize(qs_loc, scales[0])
+k8_loc = orc.quantize(np.ascontiguousarray(k_loc), scales[1])
+v8_loc = orc.quantize(np.ascontiguousarray(v_loc), scales[2])
+# 4. all-gather of K8 / V8 (padded to the largest slice), assembled in row order
+n_max = max(shard_range(N, G, g)[1] - shard_range(N, G, g)[0] for g in range(G))
+pad = lambda x: torch.from_numpy(np.pad(x, ((0, 0), (0, 0), (0, n_max - n_r), (0, 0))))
+gathered = []
+for x in (k8_loc, v8_loc):
+    parts = [torch.empty((B, H, n_max, 64), dtype=torch.uint8) for _ in range(G)]
+    dist.all_gather(parts, pad(x))
+    gathered.append(np.concatenate([p.numpy()[:, :, :shard_range(N, G, g)[1] - shard_range(N, G, g)[0]]
+                                    for g, p in enumerate(parts)], axis=2))
+k8, v8 = gathered
+# 5. this rank's rows against all keys
+o16, o, _ = orc.attention(q8_loc, k8, v8, scales[0], scales[1], scales[2])
+# the one-process oracle, on the full data
+ref = orc.layer(inp["q"], inp["k"], inp["v"], N, inp["c_h"], inp["gate"])
+ok = dict(scales=bool((scales[0] == ref["s_q"]).all() and (scales[1] == ref["s_k"]).all()
+                      and (scales[2] == ref["s_v"]).all()),
+          k8=bool((k8 == ref["k8"]).all()), v8=bool((v8 == ref["v8"]).all()),
+          q8=bool((q8_loc == ref["q8"][:, :, rows]).all()),
+          out=bool((o == ref["out"][:, rows]).all() and (o16.view(np.uint16) == ref["out16"][:, rows].view(np.uint16)).all()),
+          n_rows=int(rows.size))
+print(json.dumps(ok))
+dist.destroy_process_group()
+'''
+
+
+def test_sharded_split_reproduces_the_one_process_oracle():
+    """World size 2 on gloo, the oracle doing each rank's compute: per-slice maxima
+    all-reduced with MAX, per-slice codes all-gathered, and each rank's rows attended
+    against the gathered cache reproduce the one-process oracle's scales, e4m3 codes
+    and outputs bit for bit."""
+    port = _port()
+    procs = []
+    for r in range(2):
+        env = dict(os.environ, RANK=str(r), WORLD_SIZE="2", LOCAL_RANK=str(r), MASTER_ADDR="127.0.0.1",
+                   MASTER_PORT=str(port))
+        procs.append(subprocess.Popen([sys.executable, "-c", SHARD_CHILD, ROOT], env=env, stdout=subprocess.PIPE,
+                                      stderr=subprocess.PIPE, text=True))
+    outs = [p.communicate(timeout=240) for p in procs]
+    import json
+    for p, (o, e) in zip(procs, outs):
+        assert p.returncode == 0, e[-2000:]
+    res = [json.loads(o.strip().splitlines()[-1]) for o, _ in outs]
+    for r in res:
+        assert all(r[k] for k in ("scales", "k8", "v8", "q8", "out")), res
+    assert sum(r["n_rows"] for r in res) == 745

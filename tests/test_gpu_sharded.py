@@ -1,0 +1,129 @@
+"""The row-sharded layer call (sharded.py) and its entry points on one GPU.
+
+sdm_context_amax and sdm_quantize_with_scales are compared bit for bit with the
+oracle (maxima of |Q'|, |K|, |V| over a slice; scales amax/448; e4m3 codes).
+The whole split runs with G ranks emulated as threads on one GPU, their two
+collectives done on the host between kernel launches (no kernel waits on
+another): every rank's output rows and its full FP8 cache must equal the
+one-process layer's bit for bit."""
+import threading
+
+import numpy as np
+import pytest
+import torch
+
+from fp8_quant_logscale_b200 import binding, sharded
+from fp8_quant_logscale_b200.workloads import WORKLOADS, make_inputs
+from parity import dev, host
+
+pytestmark = pytest.mark.gpu
+
+
+def _abs_max(x, rows):
+    """[B, H] fp32 max |x| over rows [0, rows) of x [B, R, H, 64] (exact)."""
+    if rows == 0:
+        return np.zeros((x.shape[0], x.shape[2]), np.float32)
+    return np.abs(x[:, :rows].astype(np.float32)).max(axis=(1, 3))
+
+
+@pytest.mark.parametrize("gated", [False, True])
+def test_context_amax_and_quantize_with_scales(cuda_lib, orc, gated):
+    N, M, H, B = 1500, 70, 3, 2
+    inp = make_inputs(WORKLOADS["icl_n128k_m1k_h8_gated" if gated else "icl_n16k_m1k_h8"], n_ctx=N, n_query=M,
+                      heads=H, batch=B)
+    g = inp["gate"] if gated else None
+    c0, c1 = 400, 1100                       # a slice of the context rows
+    q_loc = np.ascontiguousarray(np.concatenate([inp["q"][:, c0:c1], inp["q"][:, N:N + M]], axis=1))
+    g_loc = None if g is None else np.ascontiguousarray(np.concatenate([g[:, c0:c1], g[:, N:N + M]], axis=1))
+    k_loc, v_loc = np.ascontiguousarray(inp["k"][:, c0:c1]), np.ascontiguousarray(inp["v"][:, c0:c1])
+    n_r = c1 - c0
+    amax = binding.context_amax(dev(q_loc), dev(k_loc), dev(v_loc), n_r, N, dev(inp["c_h"]), dev(g_loc))
+    qs_loc = orc.qscale(q_loc, N, inp["c_h"], g_loc)                # query scaling with the global n = N
+    want = np.stack([_abs_max(qs_loc, n_r), _abs_max(k_loc, n_r), _abs_max(v_loc, n_r)])
+    assert (host(amax) == want).all()
+    # with the full context's maxima, the slice's scales and codes are the one-process ones
+    qs = orc.qscale(inp["q"], N, inp["c_h"], g)
+    full = np.stack([_abs_max(qs, N), _abs_max(inp["k"], N), _abs_max(inp["v"], N)])
+    q8, k8, v8t, scales = binding.quantize_with_scales(dev(q_loc), dev(k_loc), dev(v_loc), n_r, N, dev(full),
+                                                       dev(inp["c_h"]), dev(g_loc), ld_k=n_r + 5)
+    s_q, s_k, s_v = (orc.context_scales(x, N) for x in (qs, inp["k"], inp["v"]))
+    sc = host(scales)
+    assert (sc[0] == s_q).all() and (sc[1] == s_k).all() and (sc[2] == s_v).all()
+    assert (host(q8) == orc.quantize(qs_loc, s_q)).all()
+    assert (host(k8)[:, :, :n_r] == orc.quantize(k_loc, s_k)).all()
+    v8 = orc.quantize(v_loc, s_v)
+    assert (host(v8t)[..., :n_r] == v8.transpose(0, 1, 3, 2)).all() and not host(v8t)[..., n_r:].any()
+
+
+def test_empty_slice_gives_zero_maxima(cuda_lib):
+    q = torch.zeros((1, 5, 2, 64), dtype=torch.float16, device="cuda")
+    amax = binding.context_amax(q, None, None, 0, 100, torch.ones(2, device="cuda"))
+    assert not amax.any()
+
+
+class _ThreadComm:
+    """G ranks as threads of one process on one GPU: the collectives meet on the host."""
+
+    def __init__(self, world, rank, shared):
+        self.world, self.rank, self.shared = world, rank, shared
+
+    def _exchange(self, t):
+        torch.cuda.synchronize()
+        self.shared["slots"][self.rank] = t.clone()
+        torch.cuda.synchronize()
+        self.shared["barrier"].wait()
+        got = torch.stack(self.shared["slots"])
+        self.shared["barrier"].wait()
+        return got
+
+    def all_reduce_max_(self, t):
+        t.copy_(self._exchange(t).amax(0))
+
+    def all_gather(self, t):
+        return self._exchange(t)
+
+
+def _run_ranks(G, inp, gated):
+    N, M = inp["N"], inp["M"]
+    shared = dict(barrier=threading.Barrier(G), slots=[None] * G)
+    results, errors = [None] * G, []
+
+    def rank_main(r):
+        try:
+            c0, c1 = sharded.shard_range(N, G, r)
+            q0, q1 = sharded.shard_range(M, G, r)
+            rows = np.r_[c0:c1, N + q0:N + q1]
+            q_loc = dev(np.ascontiguousarray(inp["q"][:, rows]))
+            g_loc = dev(np.ascontiguousarray(inp["gate"][:, rows])) if gated else None
+            out, cache = sharded.sharded_icl_attention(q_loc, dev(np.ascontiguousarray(inp["k"][:, c0:c1])),
+                                                       dev(np.ascontiguousarray(inp["v"][:, c0:c1])), N, M,
+                                                       dev(inp["c_h"]), _ThreadComm(G, r, shared), g_loc)
+            torch.cuda.synchronize()
+            results[r] = (rows, host(out), host(cache.k8), host(cache.v8t), host(cache.scales))
+        except BaseException as e:   # noqa: BLE001 -- reported by the test thread
+            errors.append(e)
+            shared["barrier"].abort()
+
+    threads = [threading.Thread(target=rank_main, args=(r,)) for r in range(G)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=300)
+    assert not errors, errors
+    return results
+
+
+@pytest.mark.parametrize("G,N,M,gated", [(2, 3000, 200, False), (3, 2049, 130, True), (4, 1000, 3, False),
+                                         (8, 9000, 1024, False)])
+def test_sharded_layer_equals_one_process(cuda_lib, G, N, M, gated):
+    H, B = 4, 1
+    inp = make_inputs(WORKLOADS["icl_n128k_m1k_h8_gated" if gated else "icl_n16k_m1k_h8"], n_ctx=N, n_query=M,
+                      heads=H, batch=B)
+    g = inp["gate"] if gated else None
+    cache = cuda_lib.FP8Cache(B, N, H, "cuda")
+    want = host(cuda_lib.icl_attention(dev(inp["q"]), dev(inp["k"]), dev(inp["v"]), N, dev(inp["c_h"]), dev(g),
+                                       cache=cache))
+    k8, v8t, sc = host(cache.k8), host(cache.v8t), host(cache.scales)
+    for rows, out, rk8, rv8t, rsc in _run_ranks(G, inp, gated):
+        assert np.array_equal(out.view(np.uint16), want[:, rows].view(np.uint16))
+        assert np.array_equal(rk8, k8) and np.array_equal(rv8t, v8t) and np.array_equal(rsc, sc)
