@@ -147,27 +147,155 @@ def measured_peaks():
 
 
 # ------------------------------------------------------------ CPU oracle
-def oracle_sample(inp, n_rows: int, seed: int = 0):
+def cpu_model() -> str:
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def oracle_inputs(inp):
+    """The oracle's query scaling, scales and e4m3 codes of a workload (untimed preparation)."""
+    import oracle
+    N = inp["N"]
+    qs = oracle.qscale(inp["q"], N, inp["c_h"], inp["gate"])
+    s_q, s_k, s_v = (oracle.context_scales(x, N) for x in (qs, inp["k"], inp["v"]))
+    return dict(qs=qs, s=(s_q, s_k, s_v), q8=oracle.quantize(qs, s_q), k8=oracle.quantize(inp["k"], s_k),
+                v8=oracle.quantize(inp["v"], s_v))
+
+
+def oracle_sample(inp, n_rows: int, seed: int = 0, prep=None):
     """Time the oracle's FP8 attention (as it stands) on a bounded row sample of the workload.
 
     The quantised inputs are prepared first (untimed); the timed part is the
     attention of n_rows query rows x all heads over all context keys.
-    Returns (TFLOP/s, seconds, threads, description).
+    Returns a dict: tflops, seconds, threads, description, rows, out (the oracle's
+    outputs of those rows, [B, n, H, 64] f64) and the prepared inputs.
     """
     import oracle
     N, H = inp["N"], inp["H"]
-    qs = oracle.qscale(inp["q"], N, inp["c_h"], inp["gate"])
-    s_q, s_k, s_v = (oracle.context_scales(x, N) for x in (qs, inp["k"], inp["v"]))
-    q8 = oracle.quantize(qs, s_q)
-    k8, v8 = oracle.quantize(inp["k"], s_k), oracle.quantize(inp["v"], s_v)
+    prep = oracle_inputs(inp) if prep is None else prep
     rows = np.sort(np.random.default_rng(seed).choice(inp["N"] + inp["M"], n_rows, replace=False)).astype(np.int64)
     t0 = time.perf_counter()
-    oracle.attention(q8, k8, v8, s_q, s_k, s_v, rows=rows)
+    _, out, _ = oracle.attention(prep["q8"], prep["k8"], prep["v8"], *prep["s"], rows=rows)
     dt = time.perf_counter() - t0
     fl = attn_flops(n_rows, N, H)
-    return fl / dt / 1e12, dt, oracle.num_threads(), (
-        f"oracle FP8 attention of {n_rows} sampled rows x {H} heads over all {N} context keys "
-        f"({fl:.3g} FLOP); quantisation prepared untimed")
+    return dict(tflops=fl / dt / 1e12, seconds=dt, threads=oracle.num_threads(), rows=rows, out=out, prep=prep,
+                desc=f"oracle FP8 attention of {n_rows} sampled rows x {H} heads over all {N} context keys "
+                     f"({fl:.3g} FLOP); quantisation prepared untimed")
+
+
+def oracle_one_thread():
+    """One-thread oracle times on the two smallest workloads: the 1K one's every row, a
+    32-row sample of the 16K one (all heads, all keys)."""
+    import oracle
+    from fp8_quant_logscale_b200.workloads import WORKLOADS, make_inputs
+    res = {}
+    keep = oracle.num_threads()
+    oracle.set_num_threads(1)
+    try:
+        for name, n_rows in (("icl_n1k_m128_h4", None), ("icl_n16k_m1k_h8", 32)):
+            inp = make_inputs(WORKLOADS[name])
+            prep = oracle_inputs(inp)
+            T = inp["N"] + inp["M"]
+            rows = np.arange(T, dtype=np.int64) if n_rows is None else \
+                np.sort(np.random.default_rng(1).choice(T, n_rows, replace=False)).astype(np.int64)
+            t0 = time.perf_counter()
+            oracle.attention(prep["q8"], prep["k8"], prep["v8"], *prep["s"], rows=rows)
+            dt = time.perf_counter() - t0
+            fl = inp["B"] * attn_flops(rows.size, inp["N"], inp["H"])
+            res[name] = {"tflops": fl / dt / 1e12, "seconds": dt, "rows": int(rows.size),
+                         "sample": "every row" if n_rows is None else f"{n_rows} sampled rows"}
+    finally:
+        oracle.set_num_threads(keep)
+    return res
+
+
+def output_parity(gpu_rows, sample, inp):
+    """The bench's own GPU outputs of the oracle sample's rows against the oracle: every
+    element within max(2e-2, one fp16 ulp), with the oracle's pinned allowance where a
+    probability sits within fp32 rounding of an e4m3 midpoint, and the mean within
+    1e-3; plus the relative RMS error of 16 of the rows against exact attention."""
+    import oracle
+    ref = sample["out"]
+    d = np.abs(gpu_rows.astype(np.float64) - ref)
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** -14))) - 10)
+    limit = np.maximum(2e-2, ulp)
+    over = np.nonzero((d > limit).any(axis=(0, 2, 3)))[0]
+    ok_over = True
+    if over.size:   # only those rows need the allowance
+        p = sample["prep"]
+        _, _, allow = oracle.attention(p["q8"], p["k8"], p["v8"], *p["s"], rows=sample["rows"][over],
+                                       **oracle.FP32_AMBIGUITY)
+        ok_over = bool((d[:, over] <= limit[:, over] + allow).all())
+    sub = np.arange(min(16, sample["rows"].size))
+    exact = oracle.attention_exact(sample["prep"]["qs"], inp["k"], inp["v"], rows=sample["rows"][sub])
+    e = gpu_rows[:, sub].astype(np.float64) - exact
+    return {"rows": int(sample["rows"].size), "max_abs": float(d.max()), "mean_abs": float(d.mean()),
+            "allowance_used": int((d > limit).sum()), "within_gates": bool(ok_over and d.mean() <= 1e-3),
+            "vs_exact_rel_rms": float(np.sqrt((e ** 2).mean() / (exact ** 2).mean())),
+            "vs_exact_rows": int(sub.size),
+            "gates": "max(2e-2, 1 fp16 ulp) per element (+ the oracle's midpoint allowance), mean 1e-3; "
+                     "oracle = the layer's definition in double"}
+
+
+def timed(fn, stream, warmup: int, samples: int):
+    """CUDA-event times (ms) of `samples` calls after `warmup` untimed ones."""
+    import torch
+    times = []
+    for i in range(warmup + samples):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= warmup:
+            times.append(a.elapsed_time(b))
+    return times
+
+
+def summary_ms(times):
+    t = sorted(times)
+    return {"median": statistics.median(t), "min": t[0], "p90": t[min(len(t) - 1, int(0.9 * len(t)))],
+            "samples": len(t)}
+
+
+def per_config(device, fp8_peak):
+    """The other workloads of the layer's specification (1K, 16K, 128K gated with outliers),
+    the pages' protocol (10 warm-ups, 30 samples): the one-call layer (quantisation
+    included) and the FP8 attention kernel alone."""
+    import torch
+
+    import fp8_quant_logscale_b200 as sdm
+    from fp8_quant_logscale_b200 import binding
+    from fp8_quant_logscale_b200.workloads import WORKLOADS, make_inputs
+    stream = torch.cuda.current_stream(device)
+    res = {}
+    for name in ("icl_n1k_m128_h4", "icl_n16k_m1k_h8", "icl_n128k_m1k_h8_gated"):
+        inp = make_inputs(WORKLOADS[name])
+        B, N, M, H = inp["B"], inp["N"], inp["M"], inp["H"]
+        q, k, v, c_h = (torch.from_numpy(inp[x]).to(device) for x in ("q", "k", "v", "c_h"))
+        gate = None if inp["gate"] is None else torch.from_numpy(inp["gate"]).to(device)
+        out = torch.empty_like(q)
+        cache = sdm.FP8Cache(B, N, H, device)
+        ws = sdm.new_workspace(sdm.workspace_size(binding.OP_ICL_ATTENTION, B, N, M, H, keep_cache=True), device)
+        layer = timed(lambda: sdm.icl_attention(q, k, v, N, c_h, gate, cache=cache, out=out, ws=ws), stream, 10, 30)
+        q8, _ = sdm.fp8_quantize_context(sdm.qscale_fused(q, c_h, N, gate), k, v, N, cache=cache)
+        ws_a = sdm.new_workspace(256, device)
+        attn = timed(lambda: sdm.fp8_attention(q8, cache, out=out, ws=ws_a), stream, 10, 30)
+        if sdm.sync_status(ws)[0] or sdm.sync_status(ws_a)[0]:
+            raise RuntimeError(f"device error word set on {name}")
+        fl = B * attn_flops(N + M, N, H)
+        a = summary_ms(attn)
+        res[name] = {"layer_ms": summary_ms(layer), "attention_ms": a,
+                     "attention_tflops": fl / (a["median"] * 1e-3) / 1e12,
+                     "attention_frac_fp8": fl / (a["median"] * 1e-3) / 1e12 / fp8_peak}
+        del q, k, v, out, cache, ws, q8
+    return res
 
 
 # ------------------------------------------------------------------ ours
@@ -264,7 +392,7 @@ def run_ours(args):
         hout, hpred = torch.empty_like(hq).pin_memory(), torch.empty_like(hqq).pin_memory()
         h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hqq))
         d2h = hout.numel() * 2 + hpred.numel() * 2
-        e_steps = max(1, min(args.steps, 3))
+        e_steps = args.steps
         barrier(device)
         torch.cuda.synchronize(device)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -293,10 +421,12 @@ def run_ours(args):
     else:
         fp8_peak = 1400.0 * 2
         peak_src = "of fallback (1.4 PF bf16 sustained x 2)"
-    traffic = args.traffic
+    traffic, traffic_src = args.traffic, "--traffic argument" if args.traffic is not None else None
     if traffic is None and args.workload == DEFAULT_WORKLOAD and ATTN_TRAFFIC["bytes"] is not None \
             and attention_source_sha256() == ATTN_TRAFFIC["source_sha256"]:
         traffic = ATTN_TRAFFIC["bytes"]
+        traffic_src = ("stored: one-pass ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of the fit "
+                       "launch on this kernel source (sha256 " + ATTN_TRAFFIC["source_sha256"][:12] + ")")
     kmean = statistics.mean(kern_ms)
     achieved = attn_flops(T, N, H) / (kmean * 1e-3) / 1e12
     clocks = clk.summary()
@@ -317,7 +447,8 @@ def run_ours(args):
         "attention_kernel_ms": kmean,
         "pct_fp8_peak": 100.0 * achieved / fp8_peak, "pct_fp8_nominal": 100.0 * achieved / FP8_NOMINAL_TFLOPS,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
-                     "frac": achieved / fp8_peak, "traffic": traffic, "peak_source": peak_src,
+                     "frac": achieved / fp8_peak, "traffic": traffic, "traffic_source": traffic_src,
+                     "peak_source": peak_src,
                      "kernel": "icl_attention_kernel (FP8 attention of all rows)"},
         # warp tiles whose probabilities all round to the e4m3 zero skip their 2^x,
         # so on peaked attention this bound of the dense softmax can be exceeded
@@ -329,10 +460,19 @@ def run_ours(args):
     }
     if e2e:
         line["e2e"] = e2e
+    if world == 1 and not args.skip_configs:
+        line["per_config"] = per_config(device, fp8_peak)
     if rank == 0 and world == 1 and not args.skip_cpu:
-        val, dt, cores, desc = oracle_sample(inp, args.cpu_rows)
-        line["cpu_baseline"] = {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                                "sample": desc, "seconds": dt}
+        smp = oracle_sample(inp, args.cpu_rows)
+        got = out.cpu().numpy()[:, smp["rows"]]
+        line["parity_sample"] = output_parity(got, smp, inp)
+        full_s = B * attn_flops(T, N, H) / (smp["tflops"] * 1e12)
+        line["cpu_baseline"] = {"value": smp["tflops"], "unit": "TFLOP/s", "cores": smp["threads"], "kind": "oracle",
+                                "sample": smp["desc"], "seconds": smp["seconds"], "cpu_model": cpu_model(),
+                                "full_layer_seconds_extrapolated": full_s,
+                                "full_layer_note": "extrapolated: the full layer's FLOPs at the sample's rate "
+                                                   "(not measured)",
+                                "one_thread": oracle_one_thread()}
     if rank == 0:
         print(json.dumps(line), flush=True)
     import torch.distributed as dist
@@ -461,10 +601,8 @@ def run_reference(args):
     w = WORKLOADS[args.workload]
     inp = make_inputs(w)
     N, H = inp["N"], inp["H"]
-    qs = oracle.qscale(inp["q"], N, inp["c_h"], inp["gate"])
-    s_q, s_k, s_v = (oracle.context_scales(x, N) for x in (qs, inp["k"], inp["v"]))
-    q8 = oracle.quantize(qs, s_q)
-    k8, v8 = oracle.quantize(inp["k"], s_k), oracle.quantize(inp["v"], s_v)
+    prep = oracle_inputs(inp)
+    q8, k8, v8, (s_q, s_k, s_v) = prep["q8"], prep["k8"], prep["v8"], prep["s"]
     rng = np.random.default_rng(0)
     times = []
     for i in range(args.warmup + args.steps):
@@ -571,6 +709,7 @@ def main(argv=None):
                     help="rows of the oracle's timed sample (about 10 s of host-core work at 512K)")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-configs", action="store_true", help="leave out the per-config timings")
     ap.add_argument("--per-kernel", action="store_true",
                     help="time each step of the path alone (one JSON line per step) instead of the benchmark step")
     ap.add_argument("--prefill", action="store_true", help="time the ragged grouped-query prefill workload")

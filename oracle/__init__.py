@@ -30,6 +30,21 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 KV_TILE = 128
 
 
+# Ambiguity radius of a key's e4m3 probability code for an implementation that
+# forms the probabilities in single precision (attention()'s delta and kappa):
+#  - delta: the 2^x evaluation (an FMA-pipe polynomial erring by at most 2.71e-6
+#    relative, MUFU ex2.approx by 2^-22) with a margin;
+#  - kappa per base-2 unit of |m2| + |t_j|: the logit passes through fp32 numbers of
+#    that size -- z accumulated from 64 exact products in fp32 on a tensor core,
+#    the scale c2 (three roundings), the shifted maximum m2 and the shift t (one
+#    each) -- and a relative error e of the logit is ln2 * e in the probability;
+#    32 roundings (2^-24 each) of that size cover them with a margin of about 2.
+# Where the definition's probability lies within that distance of a rounding
+# midpoint, either neighbouring code is what a correct fp32 implementation may
+# produce; attention()'s allowance bounds the output change of any such choice.
+FP32_AMBIGUITY = dict(delta=4e-6, kappa=32 * 2.0 ** -24 * float(np.log(2.0)))
+
+
 def split_keys(n_ctx: int) -> int:
     """Chunk length of the cached-prediction split for an n_ctx-key context."""
     per = -(-n_ctx // (32 * KV_TILE)) * KV_TILE
@@ -90,6 +105,8 @@ def _declare(L):
     L.orc_attention_exact.argtypes = [_P, _P, _P, _I, _I, _I64, _I64, _I, _P, _I64, _P]
     L.orc_num_threads.restype = _I
     L.orc_num_threads.argtypes = []
+    L.orc_set_num_threads.restype = None
+    L.orc_set_num_threads.argtypes = [_I]
 
 
 def _ptr(a: np.ndarray | None):
@@ -140,6 +157,11 @@ def log_length(n: int) -> float:
 
 def num_threads() -> int:
     return int(lib().orc_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads for the following oracle calls (OpenMP)."""
+    lib().orc_set_num_threads(int(n))
 
 
 # --- the layer ----------------------------------------------------------------

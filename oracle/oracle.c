@@ -535,10 +535,13 @@ void orc_attention_exact(const uint16_t* q, const uint16_t* k, const uint16_t* v
     }
 }
 
-/* Threads the OpenMP runtime will use (for the CPU-baseline report). */
+/* Threads the OpenMP runtime will use (for the CPU-baseline report), and a
+ * setter for single-thread timings. */
 #ifdef _OPENMP
 #include <omp.h>
 int orc_num_threads(void) { return omp_get_max_threads(); }
+void orc_set_num_threads(int n) { omp_set_num_threads(n > 0 ? n : 1); }
 #else
 int orc_num_threads(void) { return 1; }
+void orc_set_num_threads(int n) { (void)n; }
 #endif

@@ -2,25 +2,20 @@
 import numpy as np
 import torch
 
+import oracle
+
 # Output gates of the layer's specification, against the oracle on the same inputs.
 MAX_ABS = 2e-2
 MEAN_ABS = 1e-3
 
 # Ambiguity radius of a key's e4m3 probability code (oracle.attention's delta and
-# kappa): the relative error of a probability that the kernel forms in single
-# precision, against the oracle's double-precision definition.
-#  - delta: the 2^x evaluation (the FMA-pipe polynomial errs by at most 2.71e-6
-#    relative, MUFU ex2.approx by 2^-22) with a margin;
-#  - kappa per base-2 unit of |m2| + |t_j|: the logit passes through fp32 numbers of
-#    that size -- z accumulated from 64 exact products in fp32 on the tensor core,
-#    the scale c2 (three roundings), the shifted maximum m2 and the shift t (one
-#    each) -- and a relative error e of the logit is ln2 * e in the probability;
-#    32 roundings (2^-24 each) of that size cover them with a margin of about 2.
-# Where the definition's probability lies within that distance of a rounding
-# midpoint, either neighbouring code is what a correct fp32 implementation may
-# produce; the oracle's allowance bounds the output change of any such choice
-# (pinned by brute-force flipping in tests/test_oracle_attention.py).
-AMB = dict(delta=4e-6, kappa=32 * 2.0 ** -24 * np.log(2.0))
+# kappa) for the kernel's single-precision probabilities: the 2^x evaluation plus
+# 32 fp32 roundings of the logit's size (see oracle.FP32_AMBIGUITY).  Where the
+# definition's probability lies within that distance of a rounding midpoint,
+# either neighbouring code is what a correct fp32 implementation may produce; the
+# oracle's allowance bounds the output change of any such choice (pinned by
+# brute-force flipping in tests/test_oracle_attention.py).
+AMB = dict(oracle.FP32_AMBIGUITY)
 
 
 def dev(a, device="cuda"):

@@ -50,3 +50,9 @@ def test_our_arm_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["gpu_launches"] > 0
     assert "sm_mhz" in d["clocks"] and "reasons" in d["clocks"]
+    for name in ("icl_n1k_m128_h4", "icl_n16k_m1k_h8", "icl_n128k_m1k_h8_gated"):
+        c = d["per_config"][name]
+        assert 0 < c["attention_ms"]["min"] <= c["attention_ms"]["median"] <= c["attention_ms"]["p90"]
+    assert d["parity_sample"]["within_gates"] and d["parity_sample"]["rows"] == 32
+    assert 0 < d["parity_sample"]["vs_exact_rel_rms"] < 1
+    assert d["cpu_baseline"]["one_thread"]["icl_n1k_m128_h4"]["tflops"] > 0
