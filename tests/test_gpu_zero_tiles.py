@@ -105,3 +105,63 @@ def test_zero_tiles_split_kv(cuda_lib, orc, n_pred):
     _, o, allow = orc.attention(qq, k8, v8, s_q, s_k, s_v, split=split, **AMB)
     stats = gate(pred, o, allow, f"zero tiles, split-KV, {n_pred} queries")
     print(f"\nzero tiles split-KV, {n_pred} queries: {stats}")
+
+
+def _unit_c2_scale():
+    """The fp32 s_k for which the kernel's c2 = fp32(s_q s_k) * fp32(log2(e)/8) is exactly 1 (s_q = 1),
+    so a logit in base-2 units is the raw dot product z."""
+    k2 = np.float32(LOG2E / 8.0)
+    sk = np.float32(1.0) / k2
+    for cand in (sk, np.nextafter(sk, np.float32(0)), np.nextafter(sk, np.float32(1e9))):
+        if np.float32(cand * k2) == np.float32(1.0):
+            return cand
+    raise AssertionError("no fp32 scale gives c2 = 1")
+
+
+def _key_row(ones, extra_code=None):
+    """64 e4m3 codes: `ones` elements of 1.0 (0x38), optionally one extra code, the rest 0."""
+    r = np.zeros(64, np.uint8)
+    r[:ones] = 0x38
+    if extra_code is not None:
+        r[ones] = extra_code
+    return r
+
+
+@pytest.mark.parametrize("rows,split", [(5, False), (300, False), (5, True), (160, True)])
+def test_skip_threshold_band(cuda_lib, orc, rows, split):
+    """Logits placed around the skip threshold, with every query row q8 = 1.0 and c2 = 1
+    (so t = z - m in base-2 units, m = 64 from key 0 in the first tile):
+      tile 1: every key at t = -10.1015625, just below -10.0625: the warps skip it (zero codes);
+      tile 2: one key at t = -9.8984375: P = 2^-9.9 > 2^-10 is computed and rounds to 2^-9;
+      tile 3: one key at t = -10.03125: above the threshold, so computed, but P <= 2^-10
+              rounds to the e4m3 zero.
+    Other keys have t = -64.  The output must equal the oracle's bit for bit."""
+    N = 512
+    assert orc.e4m3_decode(np.uint8(0x9D)) == -0.1015625 and orc.e4m3_decode(np.uint8(0x1D)) == 0.1015625
+    assert orc.e4m3_decode(np.uint8(0x90)) == -0.03125
+    k8 = np.zeros((1, 1, N, 64), np.uint8)
+    k8[0, 0, 0] = _key_row(64)                       # z = 64: the maximum
+    k8[0, 0, 128:256] = _key_row(54, 0x9D)           # z = 53.8984375
+    k8[0, 0, 256] = _key_row(54, 0x1D)               # z = 54.1015625
+    k8[0, 0, 384] = _key_row(54, 0x90)               # z = 53.96875
+    v8 = np.full((1, 1, N, 64), 0x48, np.uint8)      # 4.0: any wrongly live key shows
+    v8[0, 0, 0], v8[0, 0, 256] = 0x38, 0x40          # 1.0 and 2.0
+    sk = _unit_c2_scale()
+    one = np.ones((1, 1), np.float32)
+    s_k = np.full((1, 1), sk, np.float32)
+    q8 = np.full((1, 1, rows, 64), 0x38, np.uint8)
+    z = orc.e4m3_decode(k8[0, 0]).sum(axis=1)
+    assert z[0] == 64 and (z[128:256] == 53.8984375).all() and z[256] == 54.1015625 and z[384] == 53.96875
+    cache = cuda_lib.FP8Cache(1, N, 1, "cuda")
+    cache.k8.copy_(dev(k8))
+    v8t = np.zeros((1, 1, 64, cache.ld_v), np.uint8)
+    v8t[..., :N] = v8.transpose(0, 1, 3, 2)
+    cache.v8t.copy_(dev(v8t))
+    cache.scales.copy_(dev(np.array([1.0, sk, 1.0], np.float32).reshape(3, 1, 1)))
+    cache.struct.filled = 1
+    out = host(cuda_lib.fp8_attention(dev(q8), cache, split=split))
+    o16, o, _ = orc.attention(q8, k8, v8, one, s_k, one, split=orc.split_keys(N) if split else 0)
+    assert np.array_equal(out.view(np.uint16), o16.view(np.uint16)), (out[0, 0, 0, :4], o[0, 0, 0, :4])
+    # the live key at -9.9 contributed 2^-9 * 2.0, nothing else but key 0
+    want = (1.0 + 2.0 ** -9 * 2.0) / (1.0 + 2.0 ** -9)
+    assert np.allclose(o, want, rtol=1e-15)
