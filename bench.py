@@ -656,6 +656,74 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_sharded(args):
+    """One layer call split by rows over the ranks (fp8_quant_logscale_b200.sharded): NCCL
+    all-reduce(MAX) of the scales' maxima and all-gather of K8 / V8^T, then every rank attends
+    its rows.  value = the whole layer's FLOPs / the slowest rank's time ("scaling": "strong").
+    With one process it runs the same calls over a one-rank NCCL group."""
+    import datetime
+    import socket
+
+    import torch
+    import torch.distributed as dist
+
+    from fp8_quant_logscale_b200 import sharded
+    from fp8_quant_logscale_b200.workloads import WORKLOADS, make_inputs
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if not dist.is_initialized():
+        if world > 1:
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        else:
+            sk = socket.socket()
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+            sk.close()
+            dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                                    timeout=datetime.timedelta(seconds=300))
+    comm = sharded.ProcessGroupComm()
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w)
+    B, N, M, H = inp["B"], inp["N"], inp["M"], inp["H"]
+    c0, c1 = sharded.shard_range(N, world, rank)
+    q0, q1 = sharded.shard_range(M, world, rank)
+    rows = np.r_[c0:c1, N + q0:N + q1]
+    q_loc = torch.from_numpy(np.ascontiguousarray(inp["q"][:, rows])).to(device)
+    k_loc = torch.from_numpy(np.ascontiguousarray(inp["k"][:, c0:c1])).to(device)
+    v_loc = torch.from_numpy(np.ascontiguousarray(inp["v"][:, c0:c1])).to(device)
+    g_loc = None if inp["gate"] is None else torch.from_numpy(np.ascontiguousarray(inp["gate"][:, rows])).to(device)
+    c_h = torch.from_numpy(inp["c_h"]).to(device)
+    del inp
+    stream = torch.cuda.current_stream(device)
+    call = lambda: sharded.sharded_icl_attention(q_loc, k_loc, v_loc, N, M, c_h, comm, g_loc)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize(device)
+    dist.barrier()
+    with ClockSampler(local) as clk:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            call()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+    dist.barrier()
+    ms = reduce_max(a.elapsed_time(b) / args.steps, device)
+    flops = B * attn_flops(N + M, N, H)
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "fp8_e4m3", "data": "synthetic",
+            "config": {"workload": w.name, "n_ctx": N, "n_query": M, "heads": H, "head_dim": 64,
+                       "parallelism": f"rows split over {world} rank(s): NCCL all-reduce(MAX) of the maxima, "
+                                      "all-gather of K8/V8^T"},
+            "clocks": clk.summary()}), flush=True)
+    dist.destroy_process_group()
+
+
 def run_prefill(args):
     """The ragged grouped-query prefill workload (bf16, head dim 128) through sdm_gqa_prefill: one
     launch timed alone (median of K after W), and 100 back-to-back launches between two events, the
@@ -741,6 +809,8 @@ def main(argv=None):
     ap.add_argument("--per-kernel", action="store_true",
                     help="time each step of the path alone (one JSON line per step) instead of the benchmark step")
     ap.add_argument("--prefill", action="store_true", help="time the ragged grouped-query prefill workload")
+    ap.add_argument("--sharded", action="store_true",
+                    help="one layer call split by rows over the ranks (NCCL), instead of independent replicas")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per attention launch from an ncu capture of the current kernel")
     args = ap.parse_args(argv)
@@ -750,6 +820,8 @@ def main(argv=None):
         run_per_kernel(args)
     elif args.prefill:
         run_prefill(args)
+    elif args.sharded:
+        run_sharded(args)
     else:
         run_ours(args)
 

@@ -5,7 +5,8 @@ oracle (maxima of |Q'|, |K|, |V| over a slice; scales amax/448; e4m3 codes).
 The whole split runs with G ranks emulated as threads on one GPU, their two
 collectives done on the host between kernel launches (no kernel waits on
 another): every rank's output rows and its full FP8 cache must equal the
-one-process layer's bit for bit."""
+one-process layer's bit for bit.  The same split also runs through a real
+NCCL process group of one rank (the only size one GPU allows)."""
 import threading
 
 import numpy as np
@@ -127,3 +128,47 @@ def test_sharded_layer_equals_one_process(cuda_lib, G, N, M, gated):
     for rows, out, rk8, rv8t, rsc in _run_ranks(G, inp, gated):
         assert np.array_equal(out.view(np.uint16), want[:, rows].view(np.uint16))
         assert np.array_equal(rk8, k8) and np.array_equal(rv8t, v8t) and np.array_equal(rsc, sc)
+
+
+NCCL_CHILD = r'''
+import os, sys, datetime
+sys.path.insert(0, sys.argv[1])
+import numpy as np, torch, torch.distributed as dist
+from fp8_quant_logscale_b200 import binding, sharded
+from fp8_quant_logscale_b200.workloads import WORKLOADS, make_inputs
+dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+torch.cuda.set_device(0)
+N, M, H = 5000, 300, 4
+inp = make_inputs(WORKLOADS["icl_n128k_m1k_h8_gated"], n_ctx=N, n_query=M, heads=H)
+d = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+out, cache = sharded.sharded_icl_attention(d(inp["q"]), d(inp["k"]), d(inp["v"]), N, M, d(inp["c_h"]),
+                                           sharded.ProcessGroupComm(), d(inp["gate"]))
+ref_cache = binding.FP8Cache(1, N, H, "cuda")
+ref = binding.icl_attention(d(inp["q"]), d(inp["k"]), d(inp["v"]), N, d(inp["c_h"]), d(inp["gate"]), cache=ref_cache)
+torch.cuda.synchronize()
+ok = torch.equal(out.view(torch.int16), ref.view(torch.int16)) and torch.equal(cache.k8, ref_cache.k8) \
+    and torch.equal(cache.v8t, ref_cache.v8t) and torch.equal(cache.scales, ref_cache.scales)
+dist.destroy_process_group()
+print("NCCL_OK" if ok else "NCCL_MISMATCH")
+'''
+
+
+def test_sharded_layer_over_a_real_nccl_group(cuda_lib):
+    """The split through torch.distributed's NCCL backend (a one-rank group: this box has one
+    GPU), in a child process: the all-reduce(MAX) and all-gather calls run for real and the
+    result equals the one-process layer bit for bit."""
+    import os
+    import socket
+    import subprocess
+    import sys
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0", MASTER_ADDR="127.0.0.1",
+               MASTER_PORT=str(port), NCCL_NVLS_ENABLE="0")
+    r = subprocess.run([sys.executable, "-c", NCCL_CHILD, root], env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr[-3000:]
+    assert "NCCL_OK" in r.stdout, r.stdout[-2000:]
