@@ -20,6 +20,7 @@ STATUS_NAMES = {0: "SDM_OK", 1: "SDM_ERR_INVALID_ARG", 2: "SDM_ERR_UNSUPPORTED",
                 7: "SDM_ERR_CUDA"}
 OP_QUANTIZE_CONTEXT, OP_ICL_ATTENTION, OP_CACHED_ATTENTION, OP_ICL_ATTENTION_F16 = 0, 1, 2, 3
 OP_CACHED_ATTENTION_OFFLOAD = 4
+OP_CACHED_PARTIALS = 5
 FP8_MIN_CONTEXT = 8192
 KV_TILE = 128
 HEAD_DIM = 64
@@ -30,7 +31,8 @@ EXPORTS = ("sdm_status_string", "sdm_version", "sdm_split_keys", "sdm_cache_layo
            "sdm_cached_attention", "sdm_fp8_eligible", "sdm_icl_attention_f16", "sdm_icl_attention_ragged",
            "sdm_icl_attention_f16_ragged", "sdm_cached_attention_offload", "sdm_gqa_prefill",
            "sdm_gqa_prefill_workspace_size", "sdm_sync_status",
-           "sdm_selftest_wait_timeout", "sdm_context_amax", "sdm_quantize_with_scales", "sdm_cache_put_rows")
+           "sdm_selftest_wait_timeout", "sdm_context_amax", "sdm_quantize_with_scales", "sdm_cache_put_rows",
+           "sdm_cached_partials", "sdm_cached_combine")
 NOALLOC_MAX_BATCH_HEADS = 4096
 
 
@@ -112,6 +114,11 @@ def lib() -> ctypes.CDLL:
         L.sdm_quantize_with_scales.restype = ctypes.c_int
         L.sdm_quantize_with_scales.argtypes = [_P, _P, _P, _I32, _I64, _I64, _I32, _I32, _I64, _P, _P, _P, _P,
                                                _P, _P, _I64, _P, _I64, _P]
+        L.sdm_cached_partials.restype = ctypes.c_int
+        L.sdm_cached_partials.argtypes = [_P, _I32, _I64, _I32, _I32, ctypes.POINTER(CacheStruct), _P, _P, _I64,
+                                          _I64, _I64, _P, _P, _P, _P, _P, _SZ, _P]
+        L.sdm_cached_combine.restype = ctypes.c_int
+        L.sdm_cached_combine.argtypes = [_P, _P, _I32, _I64, _I32, _I32, ctypes.POINTER(CacheStruct), _P, _P]
         L.sdm_cache_put_rows.restype = ctypes.c_int
         L.sdm_cache_put_rows.argtypes = [ctypes.POINTER(CacheStruct), _P, _I64, _P, _I64, _I64, _I64, _P]
         _lib = L
@@ -553,3 +560,50 @@ def cache_put_rows(cache: FP8Cache, k8_rows: torch.Tensor, v8t_cols: torch.Tenso
     with torch.cuda.device(dev):
         _check(lib().sdm_cache_put_rows(ctypes.byref(cache.struct), _ptr(k8_rows), k8_rows.shape[2], _ptr(v8t_cols),
                                         v8t_cols.shape[3], int(row0), int(n), _stream(dev)), "sdm_cache_put_rows")
+
+
+# ------------------------------------------------- cached prediction by chunks
+
+def split_count(n_ctx: int) -> int:
+    """Number of split-KV chunks of cached prediction for an n_ctx-key context."""
+    return -(-int(n_ctx) // split_keys(n_ctx))
+
+
+def partial_buffers(cache: FP8Cache, n_query: int, chunks: int | None = None):
+    """Zeroed split-KV partial buffers (acc [S,B,H,M,64], (m2, l) [S,B,H,M,2]) for `chunks`
+    chunks (default: all of the cache's)."""
+    S = split_count(cache.n_ctx) if chunks is None else int(chunks)
+    dev = cache.k8.device
+    return (torch.zeros((S, cache.batch, cache.heads, n_query, HEAD_DIM), dtype=torch.float32, device=dev),
+            torch.zeros((S, cache.batch, cache.heads, n_query, 2), dtype=torch.float32, device=dev))
+
+
+def cached_partials(q: torch.Tensor, cache: FP8Cache, k8_slice: torch.Tensor, v8t_slice: torch.Tensor, c0: int,
+                    c1: int, c_h: torch.Tensor, part_acc: torch.Tensor, part_ml: torch.Tensor,
+                    gate: torch.Tensor | None = None, ws: torch.Tensor | None = None) -> None:
+    """Partials of chunks [c0, c1) from the keys of those chunks only (sdm_cached_partials):
+    k8_slice [B,H,n,64], v8t_slice [B,H,64,ld]; writes part_acc / part_ml rows c0..c1-1."""
+    _want(q, torch.float16, "q", 4)
+    _want(k8_slice, torch.uint8, "k8_slice", 4)
+    _want(v8t_slice, torch.uint8, "v8t_slice", 4)
+    B, M, H, d = q.shape
+    dev = q.device
+    ws = new_workspace(workspace_size(OP_CACHED_PARTIALS, B, cache.n_ctx, M, H), dev) if ws is None else ws
+    with torch.cuda.device(dev):
+        _check(lib().sdm_cached_partials(_ptr(q), B, M, H, d, ctypes.byref(cache.struct), _ptr(k8_slice),
+                                         _ptr(v8t_slice), v8t_slice.shape[3], int(c0), int(c1), _ptr(c_h),
+                                         _ptr(gate), _ptr(part_acc), _ptr(part_ml), _ptr(ws), ws.numel(),
+                                         _stream(dev)), "sdm_cached_partials")
+
+
+def cached_combine(part_acc: torch.Tensor, part_ml: torch.Tensor, cache: FP8Cache, n_query: int,
+                   out: torch.Tensor | None = None) -> torch.Tensor:
+    """The fixed-order combine of all chunks' partials (sdm_cached_combine): out [B,M,H,64] fp16."""
+    dev = part_acc.device
+    out = torch.empty((cache.batch, n_query, cache.heads, HEAD_DIM), dtype=torch.float16, device=dev) \
+        if out is None else out
+    with torch.cuda.device(dev):
+        _check(lib().sdm_cached_combine(_ptr(part_acc), _ptr(part_ml), cache.batch, int(n_query), cache.heads,
+                                        HEAD_DIM, ctypes.byref(cache.struct), _ptr(out), _stream(dev)),
+               "sdm_cached_combine")
+    return out

@@ -122,6 +122,7 @@ WsLayout ws_layout(sdm_op op, int32_t B, int64_t N, int64_t M, int32_t H, int32_
     return w;
   }
   const int64_t rows = (op == SDM_OP_ICL_ATTENTION) ? N + M : M;  // cached ops: the M query rows
+  // (SDM_OP_CACHED_PARTIALS: error word, gate factors and Q8 only -- the caller owns the partials)
   w.gate_w = off;  // GatedLogScale factors, one fp16 per (row, head)
   off = align_up(off + BH * (size_t)rows * sizeof(uint16_t), kAlign);
   w.q8 = off;
@@ -296,7 +297,7 @@ sdm_status sdm_cache_layout(int32_t B, int64_t N, int32_t H, int32_t d, size_t* 
 
 size_t sdm_workspace_size(sdm_op op, int32_t B, int64_t N, int64_t M, int32_t H, int32_t d, int32_t keep_cache) {
   if (op != SDM_OP_QUANTIZE_CONTEXT && op != SDM_OP_ICL_ATTENTION && op != SDM_OP_CACHED_ATTENTION &&
-      op != SDM_OP_ICL_ATTENTION_F16 && op != SDM_OP_CACHED_ATTENTION_OFFLOAD)
+      op != SDM_OP_ICL_ATTENTION_F16 && op != SDM_OP_CACHED_ATTENTION_OFFLOAD && op != SDM_OP_CACHED_PARTIALS)
     return 0;
   if (check_shape(B, N, M, H, d) != SDM_OK || N < 1) return 0;
   return ws_layout(op, B, N, M, H, keep_cache).total;
@@ -767,6 +768,110 @@ sdm_status sdm_gqa_prefill(const void* q, const void* k, const void* v, const in
   SDM_TRY(check_ws(ws, ws_bytes, gqa_prefill_ws_bytes(seqs.data(), batch, q_heads, kv_heads, causal), dev));
   SDM_CUDA(launch_gqa_prefill(q, k, v, total_q, total_kv, seqs.data(), batch, q_heads, kv_heads, causal, out,
                               reinterpret_cast<uint8_t*>(ws), as_stream(stream)));
+  return SDM_OK;
+}
+
+// ---------------------------------------------------------------- step 4 by chunk ranges
+// The cache descriptor without its K8 / V8^T buffers: shape, state, device and
+// the scales block.
+static sdm_status check_cache_meta(const sdm_fp8_cache* c, int32_t B, int32_t H, int32_t d, int dev) {
+  if (c == nullptr) return SDM_ERR_INVALID_ARG;
+  if (c->batch != B || c->heads != H || c->head_dim != d || c->device != dev || c->n_ctx < 1 ||
+      c->ld_v != round_up(c->n_ctx, kKvTile) || (c->ragged != 0 && c->ragged != 1) || c->filled != 1)
+    return SDM_ERR_CACHE_MISMATCH;
+  if (c->scales == nullptr || !aligned(c->scales, 16)) return SDM_ERR_INVALID_ARG;
+  if (!on_device(c->scales, dev)) return SDM_ERR_CACHE_MISMATCH;
+  return SDM_OK;
+}
+
+sdm_status sdm_cached_partials(const void* q, int32_t B, int64_t M, int32_t H, int32_t d, const sdm_fp8_cache* cache,
+                               const uint8_t* k8_slice, const uint8_t* v8t_slice, int64_t ld_slice, int64_t c0,
+                               int64_t c1, const float* c_h, const void* gate, float* part_acc, float* part_ml,
+                               void* ws, size_t ws_bytes, void* stream) {
+  if (cache == nullptr) return SDM_ERR_INVALID_ARG;
+  SDM_TRY(check_shape(B, cache->n_ctx, M, H, d));
+  const int dev = current_device();
+  if (dev < 0) return SDM_ERR_CUDA;
+  SDM_TRY(check_cache_meta(cache, B, H, d, dev));
+  const int64_t N = cache->n_ctx;
+  const int64_t L = split_keys_for(N);
+  const int64_t S = n_splits_for(N);
+  if (c0 < 0 || c1 <= c0 || c1 > S) return SDM_ERR_INVALID_ARG;
+  const int64_t n = (c1 * L < N ? c1 * L : N) - c0 * L;  // keys of the slice
+  if (ld_slice < n || ld_slice % kKvTile != 0 || ld_slice > ((int64_t)1 << 30)) return SDM_ERR_INVALID_ARG;
+  if (c_h == nullptr || !aligned(c_h, 4)) return SDM_ERR_INVALID_ARG;
+  if (!on_device(c_h, dev)) return SDM_ERR_DEVICE_MISMATCH;
+  if (M == 0) return SDM_OK;
+  SDM_TRY(check_tensor(q, dev));
+  SDM_TRY(check_tensor(k8_slice, dev));
+  SDM_TRY(check_tensor(v8t_slice, dev));
+  SDM_TRY(check_tensor(part_acc, dev));
+  SDM_TRY(check_tensor(part_ml, dev));
+  if (gate != nullptr) {
+    if (!aligned(gate, 2)) return SDM_ERR_INVALID_ARG;
+    if (!on_device(gate, dev)) return SDM_ERR_DEVICE_MISMATCH;
+  }
+  const WsLayout w = ws_layout(SDM_OP_CACHED_PARTIALS, B, N, M, H, 1);
+  SDM_TRY(check_ws(ws, ws_bytes, w.total, dev));
+  cudaStream_t st = as_stream(stream);
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  uint8_t* q8 = base + w.q8;
+  // queries: scaled with the cache's n (n_b if ragged), quantised with its s_q
+  const float* meta = cache->scales + 3 * (int64_t)B * H;
+  RowsDesc dq{reinterpret_cast<const __half*>(q), B, H, M};
+  QScale qs = make_qscale(N, c_h, gate);
+  if (cache->ragged) qs.lam_b = meta + B;
+  SDM_CUDA(prepare_gate(qs, (int64_t)B * M * H, base, w, st));
+  SDM_CUDA(launch_quantize_rows(dq, qs, M, cache->scales, q8, M, nullptr, 0, st));
+  AttnArgs a;
+  a.B = B;
+  a.H = H;
+  a.T = M;
+  a.N = N;
+  a.ld_v = ld_slice;
+  a.kv_rows = n;
+  a.key_base = c0 * L;
+  a.split_base = c0;
+  a.scales = cache->scales;
+  a.partial = true;
+  a.n_splits = c1 - c0;
+  a.split_keys = L;
+  a.out = nullptr;
+  a.part_acc = part_acc;
+  a.part_ml = part_ml;
+  a.err = reinterpret_cast<uint32_t*>(base);
+  a.n_keys = cache->ragged ? reinterpret_cast<const int32_t*>(meta) : nullptr;
+  a.pad_rows = false;
+  SDM_CUDA(launch_attention(q8, k8_slice, v8t_slice, a, st));
+  return SDM_OK;
+}
+
+sdm_status sdm_cached_combine(const float* part_acc, const float* part_ml, int32_t B, int64_t M, int32_t H, int32_t d,
+                              const sdm_fp8_cache* cache, void* out, void* stream) {
+  if (cache == nullptr) return SDM_ERR_INVALID_ARG;
+  SDM_TRY(check_shape(B, cache->n_ctx, M, H, d));
+  const int dev = current_device();
+  if (dev < 0) return SDM_ERR_CUDA;
+  SDM_TRY(check_cache_meta(cache, B, H, d, dev));
+  if (M == 0) return SDM_OK;
+  SDM_TRY(check_tensor(part_acc, dev));
+  SDM_TRY(check_tensor(part_ml, dev));
+  SDM_TRY(check_tensor(out, dev));
+  AttnArgs a;
+  a.B = B;
+  a.H = H;
+  a.T = M;
+  a.N = cache->n_ctx;
+  a.ld_v = cache->ld_v;
+  a.scales = cache->scales;
+  a.partial = true;
+  a.n_splits = n_splits_for(cache->n_ctx);
+  a.split_keys = split_keys_for(cache->n_ctx);
+  a.out = reinterpret_cast<__half*>(out);
+  a.part_acc = const_cast<float*>(part_acc);
+  a.part_ml = const_cast<float*>(part_ml);
+  a.err = nullptr;
+  SDM_CUDA(launch_splitkv_reduce(a, as_stream(stream)));
   return SDM_OK;
 }
 

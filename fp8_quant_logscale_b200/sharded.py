@@ -20,6 +20,14 @@ one GPU and describe no multi-GPU scheme; this row split is the library's:
 A row's output depends only on its own e4m3 row, the full K8/V8 and the
 scales, so each rank's rows equal the one-process layer's bit for bit.
 
+Cached prediction can also be split by keys: with L = sdm_split_keys(N), the
+cache's S = ceil(N / L) split-KV chunks are independent until their
+fixed-order combine, so rank r keeps only the keys of chunks
+[S r/G, S (r+1)/G) (cache_key_slice), computes their partials
+(sdm_cached_partials), an all-gather brings every chunk's partials to every
+rank, and sdm_cached_combine gives the one-GPU result bit for bit
+(sharded_cached_attention).
+
 Collectives go through a small interface (`all_reduce_max_`, `all_gather`):
 `ProcessGroupComm` wraps a torch.distributed process group (NCCL on GPUs).
 No kernel reads another GPU's memory.
@@ -95,3 +103,44 @@ def sharded_icl_attention(q_loc: torch.Tensor, k_loc: torch.Tensor, v_loc: torch
     out_loc = _b.fp8_attention(q8_loc, cache) if T_r > 0 else torch.empty((B, 0, H, d), dtype=torch.float16,
                                                                          device=dev)
     return out_loc, cache
+
+
+def cache_key_slice(cache, c0: int, c1: int):
+    """Copies of the keys of split-KV chunks [c0, c1) of a filled cache: K8 rows
+    [B,H,n,64] and V8^T columns [B,H,64,ld] (ld a multiple of 128, zero past n)."""
+    N = cache.n_ctx
+    L = _b.split_keys(N)
+    k0, k1 = c0 * L, min(c1 * L, N)
+    ld = -(-(k1 - k0) // _b.KV_TILE) * _b.KV_TILE
+    k8 = cache.k8[:, :, k0:k1].contiguous()
+    v8t = torch.zeros((cache.batch, cache.heads, _b.HEAD_DIM, ld), dtype=torch.uint8, device=cache.k8.device)
+    v8t[..., :k1 - k0].copy_(cache.v8t[..., k0:k1])
+    return k8, v8t
+
+
+def sharded_cached_attention(queries: torch.Tensor, cache, k8_slice: torch.Tensor, v8t_slice: torch.Tensor,
+                             c_h: torch.Tensor, comm, gate: torch.Tensor | None = None) -> torch.Tensor:
+    """Cached prediction of all M queries with the cache's keys split by chunk over the ranks.
+
+    queries [B, M, H, 64] fp16 (the same on every rank); cache: the filled cache's
+    descriptor (its scales block on this device; its K8 / V8^T are not read);
+    k8_slice / v8t_slice: this rank's chunks [S r/G, S (r+1)/G) (cache_key_slice).
+    Returns out [B, M, H, 64] fp16 on every rank, equal to cached_attention's bit for bit.
+    """
+    G, r = comm.world, comm.rank
+    S = _b.split_count(cache.n_ctx)
+    M = queries.shape[1]
+    c0, c1 = shard_range(S, G, r)
+    cmax = max(shard_range(S, G, g)[1] - shard_range(S, G, g)[0] for g in range(G))
+    # room for G * cmax >= S chunks, so every rank's block [c0, c0 + cmax) lies inside
+    acc, ml = _b.partial_buffers(cache, M, chunks=G * cmax)
+    if c1 > c0:
+        _b.cached_partials(queries, cache, k8_slice, v8t_slice, c0, c1, c_h, acc, ml, gate)
+    acc_all = comm.all_gather(acc[c0:c0 + cmax])
+    ml_all = comm.all_gather(ml[c0:c0 + cmax])
+    full_acc, full_ml = _b.partial_buffers(cache, M)
+    for g in range(G):
+        g0, g1 = shard_range(S, G, g)
+        full_acc[g0:g1].copy_(acc_all[g, :g1 - g0])
+        full_ml[g0:g1].copy_(ml_all[g, :g1 - g0])
+    return _b.cached_combine(full_acc, full_ml, cache, M)

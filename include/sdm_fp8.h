@@ -65,7 +65,8 @@ typedef enum {
   SDM_OP_ICL_ATTENTION = 1,
   SDM_OP_CACHED_ATTENTION = 2,
   SDM_OP_ICL_ATTENTION_F16 = 3,
-  SDM_OP_CACHED_ATTENTION_OFFLOAD = 4
+  SDM_OP_CACHED_ATTENTION_OFFLOAD = 4,
+  SDM_OP_CACHED_PARTIALS = 5
 } sdm_op;
 
 /* Keys per online-softmax block (blocks start at key 0, or at the chunk start
@@ -422,6 +423,42 @@ sdm_status sdm_quantize_with_scales(const void* q, const void* k, const void* v,
  */
 sdm_status sdm_cache_put_rows(sdm_fp8_cache* cache, const uint8_t* k8_rows, int64_t ld_k, const uint8_t* v8t_cols,
                               int64_t ld_v, int64_t row0, int64_t n, void* stream);
+
+/*
+ * Step 4 with the cache's keys split over ranks by split-KV chunk.  Cached
+ * prediction cuts the N keys into S = ceil(N / L) chunks of L =
+ * sdm_split_keys(N) keys, computes a partial (m2, l, acc) per chunk, and
+ * combines the partials in chunk order ("[FP8 3/4] ...", opening section:
+ * "Cache chunking ... supported"; the split over ranks is the library's).
+ * Chunks are independent until the combine, so a rank holding only the keys
+ * of chunks [c0, c1) computes their partials alone; an all-gather brings all S
+ * partials to every rank, and sdm_cached_combine gives the one-GPU
+ * sdm_cached_attention result bit for bit.
+ *
+ * sdm_cached_partials: the partials of chunks [c0, c1), 0 <= c0 < c1 <= S.
+ *   cache      the full cache's descriptor (n_ctx = N, batch, heads, device,
+ *              ragged, filled, the scales block on this device); its k8 and
+ *              v8t are not read
+ *   k8_slice   [B][H][n][d] e4m3: keys [c0 L, c0 L + n) of every (b, h),
+ *              n = min(c1 L, N) - c0 L
+ *   v8t_slice  [B][H][d][ld_slice] e4m3: the same keys of V8^T; ld_slice a
+ *              multiple of 128, >= n; columns [n, ld_slice) zero
+ *   q, c_h, gate  as for sdm_cached_attention (M query rows)
+ *   part_acc   [S][B][H][M][d] fp32 and part_ml [S][B][H][M][2] fp32 (m2, l):
+ *              the rows of chunks [c0, c1) are written, the others untouched
+ *   ws         >= sdm_workspace_size(SDM_OP_CACHED_PARTIALS, B, N, M, H, d, 0)
+ * sdm_cached_combine: out [B][M][H][d] fp16 from the partials of all S chunks.
+ * Errors: SDM_ERR_INVALID_ARG (chunk range, slice sizes, null or misaligned
+ * pointers), SDM_ERR_CACHE_MISMATCH (descriptor), SDM_ERR_WORKSPACE,
+ * SDM_ERR_DEVICE_MISMATCH, SDM_ERR_UNSUPPORTED; before any work is enqueued.
+ */
+sdm_status sdm_cached_partials(const void* q, int32_t batch, int64_t n_query, int32_t heads, int32_t head_dim,
+                               const sdm_fp8_cache* cache, const uint8_t* k8_slice, const uint8_t* v8t_slice,
+                               int64_t ld_slice, int64_t c0, int64_t c1, const float* c_h, const void* gate,
+                               float* part_acc, float* part_ml, void* ws, size_t ws_bytes, void* stream);
+sdm_status sdm_cached_combine(const float* part_acc, const float* part_ml, int32_t batch, int64_t n_query,
+                              int32_t heads, int32_t head_dim, const sdm_fp8_cache* cache, void* out,
+                              void* stream);
 
 /*
  * Wait for `stream`, then read and clear the device error word at the head of

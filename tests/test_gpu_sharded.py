@@ -5,8 +5,10 @@ oracle (maxima of |Q'|, |K|, |V| over a slice; scales amax/448; e4m3 codes).
 The whole split runs with G ranks emulated as threads on one GPU, their two
 collectives done on the host between kernel launches (no kernel waits on
 another): every rank's output rows and its full FP8 cache must equal the
-one-process layer's bit for bit.  The same split also runs through a real
-NCCL process group of one rank (the only size one GPU allows)."""
+one-process layer's bit for bit.  Cached prediction with the keys split by
+split-KV chunk over the ranks equals the one-GPU cached prediction bit for bit.
+Both splits also run through a real NCCL process group of one rank (the only
+size one GPU allows)."""
 import threading
 
 import numpy as np
@@ -84,23 +86,14 @@ class _ThreadComm:
         return self._exchange(t)
 
 
-def _run_ranks(G, inp, gated):
-    N, M = inp["N"], inp["M"]
+def _threads(G, fn):
+    """fn(rank, comm) on G threads; returns the per-rank results."""
     shared = dict(barrier=threading.Barrier(G), slots=[None] * G)
     results, errors = [None] * G, []
 
     def rank_main(r):
         try:
-            c0, c1 = sharded.shard_range(N, G, r)
-            q0, q1 = sharded.shard_range(M, G, r)
-            rows = np.r_[c0:c1, N + q0:N + q1]
-            q_loc = dev(np.ascontiguousarray(inp["q"][:, rows]))
-            g_loc = dev(np.ascontiguousarray(inp["gate"][:, rows])) if gated else None
-            out, cache = sharded.sharded_icl_attention(q_loc, dev(np.ascontiguousarray(inp["k"][:, c0:c1])),
-                                                       dev(np.ascontiguousarray(inp["v"][:, c0:c1])), N, M,
-                                                       dev(inp["c_h"]), _ThreadComm(G, r, shared), g_loc)
-            torch.cuda.synchronize()
-            results[r] = (rows, host(out), host(cache.k8), host(cache.v8t), host(cache.scales))
+            results[r] = fn(r, _ThreadComm(G, r, shared))
         except BaseException as e:   # noqa: BLE001 -- reported by the test thread
             errors.append(e)
             shared["barrier"].abort()
@@ -112,6 +105,24 @@ def _run_ranks(G, inp, gated):
         t.join(timeout=300)
     assert not errors, errors
     return results
+
+
+def _run_ranks(G, inp, gated):
+    N, M = inp["N"], inp["M"]
+
+    def rank_main(r, comm):
+        c0, c1 = sharded.shard_range(N, G, r)
+        q0, q1 = sharded.shard_range(M, G, r)
+        rows = np.r_[c0:c1, N + q0:N + q1]
+        q_loc = dev(np.ascontiguousarray(inp["q"][:, rows]))
+        g_loc = dev(np.ascontiguousarray(inp["gate"][:, rows])) if gated else None
+        out, cache = sharded.sharded_icl_attention(q_loc, dev(np.ascontiguousarray(inp["k"][:, c0:c1])),
+                                                   dev(np.ascontiguousarray(inp["v"][:, c0:c1])), N, M,
+                                                   dev(inp["c_h"]), comm, g_loc)
+        torch.cuda.synchronize()
+        return rows, host(out), host(cache.k8), host(cache.v8t), host(cache.scales)
+
+    return _threads(G, rank_main)
 
 
 @pytest.mark.parametrize("G,N,M,gated", [(2, 3000, 200, False), (3, 2049, 130, True), (4, 1000, 3, False),
@@ -128,6 +139,42 @@ def test_sharded_layer_equals_one_process(cuda_lib, G, N, M, gated):
     for rows, out, rk8, rv8t, rsc in _run_ranks(G, inp, gated):
         assert np.array_equal(out.view(np.uint16), want[:, rows].view(np.uint16))
         assert np.array_equal(rk8, k8) and np.array_equal(rv8t, v8t) and np.array_equal(rsc, sc)
+
+
+@pytest.mark.parametrize("G,N,M,ragged", [(2, 40000, 300, False), (3, 40000, 64, False), (5, 33000, 129, False),
+                                          (5, 3000, 7, False), (3, 9000, 40, True)])
+def test_sharded_cached_attention(cuda_lib, orc, G, N, M, ragged):
+    """Cached prediction with the cache's keys split by split-KV chunk over G ranks (threads on
+    one GPU; with N = 3000 the 3 chunks leave two of five ranks without keys): every rank's
+    combined output equals cached_attention's bit for bit, and the oracle's chunked attention
+    within the layer's gates."""
+    from parity import AMB, gate
+    H, B = 3, 2 if ragged else 1
+    inp = make_inputs(WORKLOADS["cached_n512k_m1k_h8"], n_ctx=N, n_query=M, heads=H, batch=B)
+    lens = [N, N * 2 // 3 + 5] if ragged else None
+    cache = cuda_lib.FP8Cache(B, N, H, "cuda")
+    cuda_lib.icl_attention(dev(inp["q"]), dev(inp["k"]), dev(inp["v"]), N, dev(inp["c_h"]), cache=cache,
+                           ctx_len=lens)
+    queries, c_h = dev(inp["queries"]), dev(inp["c_h"])
+    want = host(cuda_lib.cached_attention(queries, cache, c_h))
+    S = binding.split_count(N)
+
+    def rank_main(r, comm):
+        k8s, v8ts = sharded.cache_key_slice(cache, *sharded.shard_range(S, G, r))
+        out = sharded.sharded_cached_attention(queries, cache, k8s, v8ts, c_h, comm)
+        torch.cuda.synchronize()
+        return host(out)
+
+    for out in _threads(G, rank_main):
+        assert np.array_equal(out.view(np.uint16), want.view(np.uint16))
+    if not ragged:
+        N_ = inp["N"]
+        qs = orc.qscale(inp["q"], N_, inp["c_h"])
+        s_q, s_k, s_v = (orc.context_scales(x, N_) for x in (qs, inp["k"], inp["v"]))
+        q8 = orc.quantize(orc.qscale(inp["queries"], N_, inp["c_h"]), s_q)
+        _, o, allow = orc.attention(q8, orc.quantize(inp["k"], s_k), orc.quantize(inp["v"], s_v), s_q, s_k, s_v,
+                                    split=orc.split_keys(N_), **AMB)
+        gate(want, o, allow, f"sharded cached G{G} N{N}")
 
 
 NCCL_CHILD = r'''
@@ -148,6 +195,11 @@ ref = binding.icl_attention(d(inp["q"]), d(inp["k"]), d(inp["v"]), N, d(inp["c_h
 torch.cuda.synchronize()
 ok = torch.equal(out.view(torch.int16), ref.view(torch.int16)) and torch.equal(cache.k8, ref_cache.k8) \
     and torch.equal(cache.v8t, ref_cache.v8t) and torch.equal(cache.scales, ref_cache.scales)
+# cached prediction with the keys split by chunk (one rank holds them all)
+qq = d(inp["q"][:, N - 100:N])
+k8s, v8ts = sharded.cache_key_slice(cache, 0, binding.split_count(N))
+pred = sharded.sharded_cached_attention(qq, cache, k8s, v8ts, d(inp["c_h"]), sharded.ProcessGroupComm())
+ok = ok and torch.equal(pred.view(torch.int16), binding.cached_attention(qq, ref_cache, d(inp["c_h"])).view(torch.int16))
 dist.destroy_process_group()
 print("NCCL_OK" if ok else "NCCL_MISMATCH")
 '''
