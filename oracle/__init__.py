@@ -101,6 +101,9 @@ def _declare(L):
     L.orc_attention.restype = None
     L.orc_attention.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I64, _I64, _I,
                                 _P, _I64, _I64, _I64, _I, _I, _D, _D, _P, _P, _P]
+    L.orc_attention_partials.restype = None
+    L.orc_attention_partials.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I64, _I64, _I64, _I, _P, _I64, _I64, _I64,
+                                         _I64, _P, _P, _P]
     L.orc_attention_exact.restype = None
     L.orc_attention_exact.argtypes = [_P, _P, _P, _I, _I, _I64, _I64, _I, _P, _I64, _P]
     L.orc_num_threads.restype = _I
@@ -234,6 +237,40 @@ def attention(q8, k8, v8, s_q, s_k, s_v, rows=None, bc: int = KV_TILE, split: in
                         1 if quant_p else 0, ARITH[arith], float(delta), float(kappa),
                         _ptr(out16), _ptr(out), _ptr(allow))
     return out16.view(np.float16), out, allow
+
+
+def attention_partials(q8, k8_slice, v8_slice, s_q, s_k, n_ctx: int, split: int, c0: int, c1: int, rows=None):
+    """Per-chunk partial states (definition arithmetic) of chunks [c0, c1) of `split` keys,
+    from the keys of those chunks only: k8_slice / v8_slice [B,H,n_slice,d] hold keys
+    [c0 split, c0 split + n_slice) of the n_ctx.  Returns m [C,B,H,n] (natural-log units),
+    l [C,B,H,n] and acc [C,B,H,n,d]; combine_partials of all chunks is attention(split=split)."""
+    q8 = np.ascontiguousarray(q8, np.uint8)
+    k8s = np.ascontiguousarray(k8_slice, np.uint8)
+    v8s = np.ascontiguousarray(v8_slice, np.uint8)
+    B, H, T, d = q8.shape
+    rows = np.arange(T, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, np.int64)
+    C, n = c1 - c0, rows.size
+    m = np.empty((C, B, H, n))
+    l = np.empty((C, B, H, n))
+    acc = np.empty((C, B, H, n, d))
+    sq = np.ascontiguousarray(s_q, np.float32).reshape(B * H)
+    sk = np.ascontiguousarray(s_k, np.float32).reshape(B * H)
+    lib().orc_attention_partials(_ptr(q8), _ptr(k8s), _ptr(v8s), _ptr(sq), _ptr(sk), B, H, T, int(n_ctx),
+                                 k8s.shape[2], d, _ptr(rows), n, int(split), int(c0), int(c1),
+                                 _ptr(m), _ptr(l), _ptr(acc))
+    return m, l, acc
+
+
+def combine_partials(m, l, acc, s_v):
+    """The fixed-order combine of every chunk's state: M = max_s m_s, w_s = exp(m_s - M),
+    O = (sum_s w_s acc_s) s_v / (sum_s w_s l_s).  m, l [S,B,H,n], acc [S,B,H,n,d], s_v [B,H].
+    Returns O [B,n,H,d] (double)."""
+    M = m.max(axis=0)
+    w = np.where(np.isneginf(m), 0.0, np.exp(m - M))
+    L = (w * l).sum(axis=0)
+    ACC = (w[..., None] * acc).sum(axis=0)
+    o = ACC * np.asarray(s_v, np.float64)[..., None, None] / L[..., None]
+    return o.transpose(0, 2, 1, 3)
 
 
 def attention_exact(q, k, v, rows=None):

@@ -286,6 +286,7 @@ static void e4m3_neighbours(uint8_t c, double* lo_mid, double* lo_alt,
  * |dw| * |dec(v8_j[e])|, with the same rescaling as l/acc.
  */
 enum { ORC_ARITH_DEFINITION = 0, ORC_ARITH_FP32 = 1 };
+enum { KV_TILE_ORACLE = 128 };  /* the layer's online-softmax key tile */
 
 typedef struct {
     double m2;     /* running max in log2 units; -inf if no key */
@@ -491,6 +492,56 @@ void orc_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
         free(xbuf); free(tmp);
     }
     free(vmax);
+}
+
+/*
+ * The per-chunk partial states of cached prediction (definition arithmetic):
+ * for chunks [c0, c1) of `split` keys, the state each chunk ends with --
+ * m (running maximum, natural-log units), l and acc[d] -- from a slice of the
+ * keys: k8s / v8s [B][H][n_slice][d] hold keys [c0 split, c0 split + n_slice)
+ * of the N.  Outputs [c1 - c0][B][H][n_rows] (m, l) and [...][d] (acc); a chunk
+ * with no keys gives m = -inf, l = 0, acc = 0.  Combining every chunk's state in
+ * chunk order (M = max m, w = exp(m - M), L = sum w l, ACC = sum w acc,
+ * O = ACC s_v / L) is orc_attention with the same split.
+ */
+void orc_attention_partials(const uint8_t* q8, const uint8_t* k8s, const uint8_t* v8s,
+                            const float* s_q, const float* s_k,
+                            int B, int H, int64_t T, int64_t N, int64_t n_slice, int d,
+                            const int64_t* rows, int64_t n_rows, int64_t split, int64_t c0, int64_t c1,
+                            double* m_out, double* l_out, double* acc_out) {
+    init_tables();
+    int64_t nc = c1 - c0;
+    #pragma omp parallel
+    {
+        double* xbuf = (double*)malloc(sizeof(double) * (size_t)KV_TILE_ORACLE);
+        double* tmp = (double*)malloc(sizeof(double) * (size_t)(2 * d));
+        orc_partial st; st.acc = tmp; st.amb1 = tmp + d;
+        #pragma omp for schedule(dynamic, 1)
+        for (int64_t task = 0; task < (int64_t)B * H * n_rows * nc; ++task) {
+            int64_t c = task % nc, rest = task / nc;
+            int64_t ri = rest % n_rows, bh = rest / n_rows;
+            const uint8_t* qrow = q8 + (bh * T + rows[ri]) * d;
+            const uint8_t* kb = k8s + bh * n_slice * d;
+            const uint8_t* vb = v8s + bh * n_slice * d;
+            int64_t jb = (c0 + c) * split, je = jb + split < N ? jb + split : N;
+            double scale = (double)s_q[bh] * (double)s_k[bh] / sqrt((double)d);
+            int64_t o = (c * B * H + bh) * n_rows + ri;
+            if (je <= jb) {
+                m_out[o] = -INFINITY; l_out[o] = 0.0;
+                for (int e = 0; e < d; ++e) acc_out[o * d + e] = 0.0;
+                continue;
+            }
+            /* keys [jb, je) are slice keys [jb - c0 split, je - c0 split); tiles are
+             * aligned to the chunk start either way */
+            int64_t off = c0 * split;
+            attend_range_definition(qrow, kb, vb, jb - off, je - off, d, scale, KV_TILE_ORACLE, 1,
+                                    0.0, 0.0, &st, xbuf);
+            m_out[o] = st.m2 / kLog2e;
+            l_out[o] = st.l;
+            for (int e = 0; e < d; ++e) acc_out[o * d + e] = st.acc[e];
+        }
+        free(xbuf); free(tmp);
+    }
 }
 
 /*

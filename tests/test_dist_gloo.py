@@ -130,3 +130,66 @@ def test_sharded_split_reproduces_the_one_process_oracle():
     for r in res:
         assert all(r[k] for k in ("scales", "k8", "v8", "q8", "out")), res
     assert sum(r["n_rows"] for r in res) == 745
+
+
+CACHED_CHILD = r'''
+import os, sys, json
+sys.path.insert(0, sys.argv[1])
+import numpy as np
+import torch
+import torch.distributed as dist
+import oracle as orc
+from fp8_quant_logscale_b200.sharded import shard_range
+from fp8_quant_logscale_b200.workloads import WORKLOADS, make_inputs
+
+dist.init_process_group("gloo")
+G, r = dist.get_world_size(), dist.get_rank()
+N, M, H, B = 5000, 37, 2, 1
+inp = make_inputs(WORKLOADS["cached_n512k_m1k_h8"], n_ctx=N, n_query=M, heads=H, batch=B)
+qs = orc.qscale(inp["q"], N, inp["c_h"])
+s_q, s_k, s_v = (orc.context_scales(x, N) for x in (qs, inp["k"], inp["v"]))
+k8, v8 = orc.quantize(inp["k"], s_k), orc.quantize(inp["v"], s_v)
+q8 = orc.quantize(orc.qscale(inp["queries"], N, inp["c_h"]), s_q)
+L = orc.split_keys(N)
+S = -(-N // L)
+# this rank keeps only the keys of its chunks
+c0, c1 = shard_range(S, G, r)
+k0, k1 = c0 * L, min(c1 * L, N)
+m, l, acc = orc.attention_partials(q8, k8[:, :, k0:k1], v8[:, :, k0:k1], s_q, s_k, N, L, c0, c1)
+cmax = max(shard_range(S, G, g)[1] - shard_range(S, G, g)[0] for g in range(G))
+def pad(x):
+    out = np.full((cmax,) + x.shape[1:], -np.inf if x is m else 0.0)
+    out[:x.shape[0]] = x
+    return torch.from_numpy(out)
+gathered = []
+for x in (m, l, acc):
+    parts = [torch.empty((cmax,) + x.shape[1:], dtype=torch.float64) for _ in range(G)]
+    dist.all_gather(parts, pad(x))
+    gathered.append(np.concatenate([p.numpy()[:shard_range(S, G, g)[1] - shard_range(S, G, g)[0]]
+                                    for g, p in enumerate(parts)], axis=0))
+got = orc.combine_partials(*gathered, s_v)
+_, want, _ = orc.attention(q8, k8, v8, s_q, s_k, s_v, split=L)
+print(json.dumps({"chunks": int(c1 - c0), "S": int(S),
+                  "rel": float(np.abs(got - want).max() / np.abs(want).max())}))
+dist.destroy_process_group()
+'''
+
+
+def test_cached_chunk_split_reproduces_the_one_process_oracle():
+    """World size 2 on gloo, the oracle doing each rank's compute: each rank keeps only the keys
+    of its split-KV chunks and computes their partial states; all-gathered and combined in chunk
+    order they give the one-process oracle's cached prediction (to double rounding)."""
+    port = _port()
+    procs = []
+    for r in range(2):
+        env = dict(os.environ, RANK=str(r), WORLD_SIZE="2", LOCAL_RANK=str(r), MASTER_ADDR="127.0.0.1",
+                   MASTER_PORT=str(port))
+        procs.append(subprocess.Popen([sys.executable, "-c", CACHED_CHILD, ROOT], env=env, stdout=subprocess.PIPE,
+                                      stderr=subprocess.PIPE, text=True))
+    outs = [p.communicate(timeout=240) for p in procs]
+    import json
+    for p, (o, e) in zip(procs, outs):
+        assert p.returncode == 0, e[-2000:]
+    res = [json.loads(o.strip().splitlines()[-1]) for o, _ in outs]
+    assert sum(x["chunks"] for x in res) == res[0]["S"] >= 2
+    assert all(x["rel"] <= 1e-12 for x in res), res

@@ -353,3 +353,21 @@ def test_lossless_when_inputs_are_e4m3_values(orc):
     _, out, _ = orc.attention(q8, k8, v8, sq, sk, sv, quant_p=False)
     exact = orc.attention_exact(q, k, v)
     assert np.abs(out - exact).max() <= 1e-5 * np.abs(exact).max()
+
+
+@pytest.mark.parametrize("split,N", [(256, 700), (128, 300), (1024, 700)])
+def test_chunk_partials_combine_to_the_chunked_attention(orc, split, N):
+    """Every chunk's partial state, combined in chunk order, is the oracle's cached
+    (chunked) attention; partials computed from a key slice equal those from all keys."""
+    q8, k8, v8, sq, sk, sv = _problem(orc, T=21, N=N, seed=43, qscale=1.0)
+    S = -(-N // split)
+    m, l, acc = orc.attention_partials(q8, k8, v8, sq, sk, N, split, 0, S)
+    got = orc.combine_partials(m, l, acc, sv)
+    _, want, _ = orc.attention(q8, k8, v8, sq, sk, sv, split=split)
+    assert np.abs(got - want).max() <= 1e-12 * np.abs(want).max()
+    for c0, c1 in ((0, 1), (1, S), (S - 1, S)):
+        if c1 <= c0:
+            continue
+        k0, k1 = c0 * split, min(c1 * split, N)
+        ms, ls, accs = orc.attention_partials(q8, k8[:, :, k0:k1], v8[:, :, k0:k1], sq, sk, N, split, c0, c1)
+        assert np.array_equal(ms, m[c0:c1]) and np.array_equal(ls, l[c0:c1]) and np.array_equal(accs, acc[c0:c1])
