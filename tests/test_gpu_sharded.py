@@ -224,3 +224,39 @@ def test_sharded_layer_over_a_real_nccl_group(cuda_lib):
                        timeout=300)
     assert r.returncode == 0, r.stderr[-3000:]
     assert "NCCL_OK" in r.stdout, r.stdout[-2000:]
+
+
+def test_new_entry_points_refuse_bad_arguments(cuda_lib):
+    """Host-side checks before any work is enqueued: chunk ranges, slice pitches, row ranges,
+    slice row counts."""
+    import ctypes
+    L = binding.lib()
+    N, M, H = 3000, 8, 2
+    inp = make_inputs(WORKLOADS["cached_n512k_m1k_h8"], n_ctx=N, n_query=M, heads=H)
+    cache = cuda_lib.FP8Cache(1, N, H, "cuda")
+    cuda_lib.icl_attention(dev(inp["q"]), dev(inp["k"]), dev(inp["v"]), N, dev(inp["c_h"]), cache=cache)
+    S = binding.split_count(N)
+    q, c_h = dev(inp["queries"]), dev(inp["c_h"])
+    acc, ml = binding.partial_buffers(cache, M)
+    k8s, v8ts = sharded.cache_key_slice(cache, 0, S)
+    ws = cuda_lib.new_workspace(cuda_lib.workspace_size(binding.OP_CACHED_PARTIALS, 1, N, M, H), "cuda")
+    P = ctypes.c_void_p
+    stream = P(torch.cuda.current_stream().cuda_stream)
+
+    def partials(c0, c1, ld=v8ts.shape[3]):
+        return L.sdm_cached_partials(P(q.data_ptr()), 1, M, H, 64, ctypes.byref(cache.struct), P(k8s.data_ptr()),
+                                     P(v8ts.data_ptr()), ld, c0, c1, P(c_h.data_ptr()), None, P(acc.data_ptr()),
+                                     P(ml.data_ptr()), P(ws.data_ptr()), ws.numel(), stream)
+
+    assert partials(0, S) == 0
+    for c0, c1 in ((0, S + 1), (1, 1), (-1, 1), (2, 1)):
+        assert partials(c0, c1) == 1, (c0, c1)                         # SDM_ERR_INVALID_ARG
+    assert partials(0, S, ld=v8ts.shape[3] - 128) == 1                 # pitch below the slice's keys
+    assert partials(0, S, ld=v8ts.shape[3] + 1) == 1                   # pitch not a multiple of 128
+    assert L.sdm_cache_put_rows(ctypes.byref(cache.struct), P(k8s.data_ptr()), N, P(v8ts.data_ptr()),
+                                v8ts.shape[3], 1, N, stream) == 1     # rows [1, N + 1) outside the cache
+    amax = torch.zeros((3, 1, H), dtype=torch.float32, device="cuda")
+    qq = dev(inp["q"])
+    assert L.sdm_context_amax(P(qq.data_ptr()), P(qq.data_ptr()), P(qq.data_ptr()), 1, 10, 9, H, 64, N,
+                              P(c_h.data_ptr()), None, P(amax.data_ptr()), stream) == 1   # q_rows < n_ctx
+    torch.cuda.synchronize()
