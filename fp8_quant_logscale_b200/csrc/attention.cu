@@ -422,17 +422,19 @@ __global__ void __launch_bounds__(Cfg<kTiles>::kThreads, Cfg<kTiles>::kMinBlocks
       // zeros, or nothing if the columns already hold zeros. The P V product
       // still runs and adds exact zeros, so the result is the same to the bit.
       // (Such a tile cannot raise the running max, so m_run and m2 stay.)
-      // The arrival on p_full must not come before the previous tile's phase
-      // has completed, or a fast warp would count twice toward it: a store
-      // waits for the previous P V as the dense path does; without a store
-      // the warp waits for the previous P_t to be complete.
+      // The arrival on p_full waits, as the dense path's does, for the previous
+      // P V to be done: that MMA is issued only once the MMA thread has seen
+      // the previous p_full phase complete, so p_full never runs more than one
+      // phase ahead of the thread that waits on it by parity. (Waiting only for
+      // the previous p_full phase would let four zero-tile warps complete two
+      // phases before the MMA thread looks, which its parity wait cannot tell
+      // from none.)
       if (__all_sync(0xffffffffu, __fmaf_rn(mtile, c2, nm2) < kDeadExponent)) {
         if (it > 0) {
-          ok = p_zero ? mbar_wait(&s.p_full[t], (it - 1) & 1, abort_flag, kWaitLimit)
-                      : mbar_wait(&s.o_ready[t], (it - 1) & 1, abort_flag, kWaitLimit);
+          ok = mbar_wait(&s.o_ready[t], (it - 1) & 1, abort_flag, kWaitLimit);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) {
-            if (lane == 0) raise_abort(s, p.err, p_zero ? kErrTimeoutP : kErrTimeoutO);
+            if (lane == 0) raise_abort(s, p.err, kErrTimeoutO);
             break;
           }
           tc_fence_after();
