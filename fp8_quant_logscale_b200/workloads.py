@@ -63,6 +63,10 @@ WORKLOADS = {
     "icl_n512k_m1k_h8": Workload(
         "icl_n512k_m1k_h8", 524288, 1024, 8, seed=4,
         description="N=524288, M=1024, H=8, d=64, fp16 N(0,1); LogScale; FP8 self + cross attention"),
+    "icl_n256k_m1k_h8": Workload(
+        "icl_n256k_m1k_h8", 262144, 1024, 8, seed=9,
+        description="N=262144, M=1024, H=8, d=64, fp16 N(0,1); LogScale: the 512K workload's recipe at half "
+                    "the context, small enough for a full ncu capture of the long-context attention"),
     "icl_n128k_m1k_h8_flat": Workload(
         "icl_n128k_m1k_h8_flat", 131072, 1024, 8, head_factor=(0.01, 0.02), seed=8,
         description="N=131072, M=1024, H=8, d=64, fp16 N(0,1) scaled per (tensor, head) by U(0.01,0.02): "

@@ -138,6 +138,28 @@ def test_full_size_ragged_workload_sampled(cuda_lib, orc):
         gate(out[b:b + 1, rows_b[sel]], r["out"], r["allow"], f"full ragged batch {b} n_b={n}")
 
 
+def test_ragged_long_context_decoupled_issue(cuda_lib, orc):
+    """At 262,144 keys and more the one-call layer issues each query tile's MMAs from its
+    own warp: a ragged batch there (a ragged last key tile, padding rows, CTAs whose rows
+    are all padding) against the oracle's layer on each estimator alone, sampled rows."""
+    B, N, M, H = 2, 262144, 64, 2
+    inp = make_inputs(W, n_ctx=N, n_query=M, heads=H, batch=B)
+    inp["ctx_len"] = np.array([N, 150017], np.int64)
+    inp = poison_padding(inp)
+    out, cache = fit_ragged(cuda_lib, inp)
+    sc = host(cache.scales)
+    for b, n in enumerate(inp["ctx_len"]):
+        n = int(n)
+        assert not out[b, n:N].view(np.uint16).any(), f"padding rows of batch {b} not zero"
+        rows_b = np.r_[0:n, N:N + M]
+        sel = np.unique(np.r_[np.arange(0, n, n // 40), [1, n - 1], np.arange(n, n + M)]).astype(np.int64)
+        r = orc.layer(np.ascontiguousarray(inp["q"][b:b + 1, rows_b]), np.ascontiguousarray(inp["k"][b:b + 1, :n]),
+                      np.ascontiguousarray(inp["v"][b:b + 1, :n]), n, inp["c_h"], rows=sel, **AMB)
+        assert (sc[0][b] == r["s_q"][0]).all() and (sc[1][b] == r["s_k"][0]).all() and (sc[2][b] == r["s_v"][0]).all()
+        stats = gate(out[b:b + 1, rows_b[sel]], r["out"], r["allow"], f"long ragged batch {b} n_b={n}")
+        print(f"\nlong ragged batch {b} n_b={n}: {stats}")
+
+
 def test_precision_rule_uses_the_smallest_estimator(cuda_lib):
     inp = make_inputs(W, n_ctx=9000, n_query=16, heads=2, batch=2)
     N = inp["N"]
