@@ -16,11 +16,12 @@
 //               M=128 N=128 K=64, operands in smem) and O_t += P_t [V^T;1]^T
 //               (M=128 N=80 K=128, P read from TMEM); the 16 extra rows of
 //               ones in the V stage give the row sum l = sum P in O's
-//               columns 64..79, so the softmax never adds up P itself;
+//               columns 64..79, so the softmax never adds up P itself (the
+//               decoupled build has warps 9 and 10, one issuer per tile);
 //   warps 0..7  softmax, warpgroup t for tile t, one TMEM lane (= query row)
 //               per thread: all 128 logits of the tile read in one TMEM pass,
-//               row max, P = 2^(z*c2 - m2) -> e4m3 written back into TMEM over
-//               S, and O rescaled when the running max rises.
+//               row max, P = 2^(z*c2 - m2) -> e4m3 stored in P_t's own TMEM
+//               columns, and O rescaled when the running max rises.
 // The two tiles ping-pong: while one warpgroup turns S into P the tensor core
 // works on the other tile.
 //
