@@ -535,7 +535,7 @@ def run_per_kernel(args):
     q8 = torch.empty((B, H, T, 64), dtype=torch.uint8, device=device)
     ws_q = sdm.new_workspace(sdm.workspace_size(binding.OP_QUANTIZE_CONTEXT, B, N, M, H), device)
     ws_a = sdm.new_workspace(256, device)
-    Mq = 1024
+    Mq = args.cached_queries
     queries = q[:, :Mq].contiguous()
     pred = torch.empty_like(queries)
     ws_c = sdm.new_workspace(sdm.workspace_size(binding.OP_CACHED_ATTENTION, B, N, Mq, H), device)
@@ -557,7 +557,7 @@ def run_per_kernel(args):
          2 * 3 * el(N) + 3 * (el(T) + 2 * el(N)), 0.0),
         ("a3 FP8 attention (sdm_fp8_attention)", lambda: sdm.fp8_attention(q8, cache, out=out, ws=ws_a),
          el(T) + 2 * el(N) + 2 * el(T), B * attn_flops(T, N, H)),
-        ("a4 cached prediction, 1024 queries (sdm_cached_attention)",
+        (f"a4 cached prediction, {Mq} queries (sdm_cached_attention)",
          lambda: sdm.cached_attention(queries, cache, c_h, gate=None, out=pred, ws=ws_c),
          2 * el(Mq) + 2 * el(N) + 2 * el(Mq), B * attn_flops(Mq, N, H)),
         ("a5 fp16 attention, query scaling included (sdm_icl_attention_f16)",
@@ -592,7 +592,7 @@ def run_per_kernel(args):
     k_dst, v_dst = torch.empty_like(cache.k8), torch.empty_like(cache.v8t)
     cache_bytes = off.k8.numel() + off.v8t.numel()
     steps += [
-        ("a8 cached prediction from the host-offloaded cache, 1024 queries (sdm_cached_attention_offload)",
+        (f"a8 cached prediction from the host-offloaded cache, {Mq} queries (sdm_cached_attention_offload)",
          lambda: sdm.cached_attention_offload(queries, off, c_h, out=pred, ws=ws_o),
          cache_bytes + 2 * el(Mq) * 2, B * attn_flops(Mq, N, H)),
         ("ref: page-locked host-to-device copy of the same K8 / V8^T bytes (cudaMemcpyAsync, not this library)",
@@ -808,6 +808,8 @@ def main(argv=None):
     ap.add_argument("--skip-configs", action="store_true", help="leave out the per-config timings")
     ap.add_argument("--per-kernel", action="store_true",
                     help="time each step of the path alone (one JSON line per step) instead of the benchmark step")
+    ap.add_argument("--cached-queries", type=int, default=1024,
+                    help="--per-kernel: query rows of the cached-prediction steps (a4, a8)")
     ap.add_argument("--prefill", action="store_true", help="time the ragged grouped-query prefill workload")
     ap.add_argument("--sharded", action="store_true",
                     help="one layer call split by rows over the ranks (NCCL), instead of independent replicas")
